@@ -35,14 +35,14 @@ _CHUNK = 1 << 24  # draw at most this many normals at a time
 
 
 def _randn(shape, gen, dtype, std=1.0):
-    """randn in float32 (chunked along dim 0 in draw order), scaled, rounded to dtype."""
-    out = torch.empty(shape, dtype=dtype)
+    """randn in float32 (chunked, in draw order), scaled, rounded to dtype."""
+    out = torch.empty(shape, dtype=dtype, device=gen.device)
     flat = out.view(-1)
     n = flat.numel()
     pos = 0
     while pos < n:
         m = min(_CHUNK, n - pos)
-        x = torch.randn(m, generator=gen, dtype=torch.float32)
+        x = torch.randn(m, generator=gen, dtype=torch.float32, device=gen.device)
         if std != 1.0:
             x.mul_(std)
         flat[pos:pos + m] = x.to(dtype)
@@ -65,14 +65,16 @@ class DecodeInputs:
 
 
 def decode_inputs(B, H, G, d_h, T_cap, dtype=torch.bfloat16, seed=0, ragged=None,
-                  seqlens=None, nan_pad=True, scale=None, std=1.0):
-    """q [B,H,d_h], K/V [B,G,T_cap,d_h], seqlens [B] int32 (CPU tensors).
+                  seqlens=None, nan_pad=True, scale=None, std=1.0, device="cpu"):
+    """q [B,H,d_h], K/V [B,G,T_cap,d_h], seqlens [B] int32.
 
     ragged=(lo, hi): seqlens drawn uniform over the integers lo..hi inclusive
     after K and V.  An explicit ``seqlens`` list overrides it.  Otherwise every
-    sequence holds T_cap tokens.
+    sequence holds T_cap tokens.  device="cuda" draws from torch's CUDA
+    generator with the same seed and order (other values than on the CPU, same
+    recipe), for inputs too large to draw on the host; seqlens stay on the CPU.
     """
-    gen = torch.Generator().manual_seed(seed)
+    gen = torch.Generator(device=device).manual_seed(seed)
     q = _randn((B, H, d_h), gen, dtype, std)
     k = _randn((B, G, T_cap, d_h), gen, dtype, std)
     v = _randn((B, G, T_cap, d_h), gen, dtype, std)
@@ -80,7 +82,8 @@ def decode_inputs(B, H, G, d_h, T_cap, dtype=torch.bfloat16, seed=0, ragged=None
         sl = torch.as_tensor(seqlens, dtype=torch.int32).reshape(B)
     elif ragged is not None:
         lo, hi = ragged
-        sl = torch.randint(lo, hi + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+        sl = torch.randint(lo, hi + 1, (B,), generator=gen, dtype=torch.int64,
+                           device=gen.device).to(torch.int32).cpu()
     else:
         sl = torch.full((B,), T_cap, dtype=torch.int32)
     if nan_pad:

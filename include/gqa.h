@@ -1,0 +1,166 @@
+/*
+ * gqa.h -- C ABI of libgqa.so: grouped-query attention (GQA) on NVIDIA B200
+ * (sm_100a).
+ *
+ * Notation.  B batch, H query heads, G key/value heads with G | H, r = H/G
+ * query heads per group, d_h head dimension, T_cap cache capacity, S prompt
+ * length, d model dimension.  Query head i (0-indexed) reads KV head i / r,
+ * the 0-indexed form of g(i) = ceil(i*G/H) over 1-indexed heads
+ * ("Grouped-Query Attention", llm-arch-kb, section 2 "Derivation", "The
+ * grouping": G contiguous groups of H/G query heads).
+ *
+ * Conventions shared by every call.
+ *   - Pointers named as device pointers must point to device memory (or
+ *     memory the device can address) that stays valid until the work queued
+ *     on `stream` has finished.  Host pointers are read before the call
+ *     returns.  The library keeps no pointer after a call returns, allocates
+ *     no device memory, and owns nothing but a device status word.
+ *   - Tensors are dense and row-major in the order of their shape; no strides.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and returns a status code.  Arguments are
+ *     validated on the host before any launch; an invalid call launches
+ *     nothing and returns a negative code, with the reason available from
+ *     gqa_last_error_string() on the calling thread.
+ *   - Conditions only the device can see (a seqlens entry outside [0, T_cap],
+ *     a bounded wait that ran out) set bits of a device status word that
+ *     gqa_get_status() reads and clears.  No kernel traps.
+ *   - Results are deterministic: the same inputs and launch give the same bits.
+ */
+#ifndef GQA_H
+#define GQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GQA_API __attribute__((visibility("default")))
+#else
+#define GQA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *gqa_stream_t; /* same type as cudaStream_t */
+
+typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
+
+enum {
+    GQA_OK = 0,
+    GQA_ERR_INVALID = -1,     /* bad shape, null pointer, G does not divide H */
+    GQA_ERR_UNSUPPORTED = -2, /* valid but not built: d_h, dtype, group size  */
+    GQA_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned             */
+    GQA_ERR_CUDA = -4,        /* a CUDA runtime or driver call failed         */
+    GQA_ERR_WORKSPACE = -5,   /* workspace missing or too small               */
+    GQA_ERR_TIMEOUT = -6,     /* device: a bounded wait ran out               */
+    GQA_ERR_SEQLEN = -7       /* device: a seqlens entry was outside [0,T_cap] */
+};
+
+/*
+ * gqa_kv_cache_bytes -- bytes the KV cache grows by per token: one key and one
+ * value vector of d_h scalars for each of G KV heads in each of L layers,
+ * 2 * G * d_h * L * elem_bytes ("Grouped-Query Attention", llm-arch-kb,
+ * section 2 "KV-cache footprint"; G = H gives the MHA figure of section 1
+ * "Premise", G = 1 the MQA one).  Pure host arithmetic; returns 0 if any
+ * argument is not positive.
+ */
+GQA_API uint64_t gqa_kv_cache_bytes(int G, int d_h, int L, int elem_bytes);
+
+/*
+ * gqa_decode_workspace_bytes -- device workspace gqa_decode needs for this
+ * shape on the current device (it depends on the device's SM count).  Returns
+ * 0 for an invalid shape.  The caller allocates it (any device allocation,
+ * 256-byte aligned) and may reuse it across calls on one stream; calls that
+ * run concurrently need separate workspaces.
+ */
+GQA_API size_t gqa_decode_workspace_bytes(int B, int H, int G, int d_h, int T_cap,
+                                  gqa_dtype dt);
+
+/*
+ * gqa_decode -- one decode step of GQA attention over a KV cache: for each
+ * sequence b and query head i,
+ *     out[b,i,:] = sum_{t < T_b} softmax_t(scale * <q[b,i,:], K[b,g,t,:]>) V[b,g,t,:]
+ * with g = i / (H/G) and T_b = seqlens[b].  Every cached key and value of the
+ * sequence is read once for the new token ("Grouped-Query Attention",
+ * llm-arch-kb, section 1 "Premise"; scores, softmax over keys and the value
+ * sum as in section 3 "Reference implementation").  Pass scale = 1/sqrt(d_h)
+ * for the page's scaling.
+ *
+ *   q        device, [B, H, d_h]        dtype dt, 16-byte aligned
+ *   k_cache  device, [B, G, T_cap, d_h] dtype dt, 16-byte aligned
+ *   v_cache  device, [B, G, T_cap, d_h] dtype dt, 16-byte aligned
+ *   seqlens  device, [B] int32; entries 0 <= T_b <= T_cap.  Positions >= T_b
+ *            are never used (their contents may be anything, NaN included).
+ *            Entries outside the range are clamped and flag GQA_ERR_SEQLEN.
+ *            T_b = 0 gives a zero output row.
+ *   out      device, [B, H, d_h] dtype dt, 16-byte aligned
+ *   workspace device, >= gqa_decode_workspace_bytes(...) bytes, 256-byte
+ *            aligned; scratch for per-split partial results.
+ *   dt       GQA_BF16 (tensor-core scores and P.V, fp32 softmax/accumulate)
+ *            or GQA_F32 (fp32 CUDA-core arithmetic throughout).
+ *   Supported: d_h in {64, 128}; bf16 needs H/G <= 64.
+ * Internally: a split-KV kernel over equal shares of the cache tiles (TMA
+ * staged, fp32 online softmax per split) and a combine kernel that merges
+ * the per-split (max, sum, partial output) triples exactly.
+ */
+GQA_API int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *seqlens, float scale, void *out, int B, int H,
+               int G, int d_h, int T_cap, gqa_dtype dt, void *workspace,
+               size_t workspace_bytes, gqa_stream_t stream);
+
+/*
+ * gqa_prefill_causal -- causal GQA attention over a whole prompt: for each b,
+ * position s and query head i,
+ *     out[b,s,i,:] = sum_{t <= s} softmax_t(scale * <q[b,s,i,:], k[b,t,g,:]>) v[b,t,g,:]
+ * with g = i / (H/G) ("Grouped-Query Attention", llm-arch-kb, section 3
+ * "Reference implementation": scores over sqrt(d_h), causal mask, softmax on
+ * the key axis, K/V broadcast to the H/G heads of each group).  The mask keeps
+ * the diagonal (t = s).  Pass scale = 1/sqrt(d_h) for the page's scaling.
+ *
+ *   q    device, [B, S, H, d_h] bf16, 16-byte aligned
+ *   k, v device, [B, S, G, d_h] bf16, 16-byte aligned
+ *   out  device, [B, S, H, d_h] bf16, 16-byte aligned
+ *   Supported: dt = GQA_BF16, d_h = 128, H/G even; any S >= 1.
+ * Internally: tcgen05 tensor-core MMAs with fp32 accumulators in tensor
+ * memory, TMA-fed shared-memory tiles, fp32 online softmax, P in bf16.
+ */
+GQA_API int gqa_prefill_causal(const void *q, const void *k, const void *v, void *out,
+                       int B, int S, int H, int G, int d_h, float scale,
+                       gqa_dtype dt, gqa_stream_t stream);
+
+/*
+ * gqa_meanpool_kv -- averaging initialisation of GQA key/value projections
+ * from an MHA checkpoint: each of the G new heads is the plain mean of the H/G
+ * original heads of its group,
+ *     WK_out[g,:,:] = (sum_{j < r} WK[g*r + j,:,:]) / r,  same for WV,
+ * summed in ascending head order in binary64, divided by r, then rounded once
+ * to nearest-even in dt ("Grouped-Query Attention", llm-arch-kb, section 2
+ * "Uptraining recipe (averaging-init)").  Bit-exact with that definition.
+ *
+ *   WK, WV          device, [H, d_h, d] dtype dt
+ *   WK_out, WV_out  device, [G, d_h, d] dtype dt (must not overlap inputs)
+ *   dt              GQA_BF16 or GQA_F32; any d_h, d >= 1.
+ */
+GQA_API int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *WV_out,
+                    int H, int G, int d_h, int d, gqa_dtype dt,
+                    gqa_stream_t stream);
+
+/*
+ * gqa_get_status -- synchronises `stream`, then reads and clears the device
+ * status word: GQA_OK, GQA_ERR_SEQLEN or GQA_ERR_TIMEOUT (device-side
+ * conditions of earlier calls on this device), or GQA_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+GQA_API int gqa_get_status(gqa_stream_t stream);
+
+/* Reason for the last non-OK return on the calling thread ("" if none). */
+GQA_API const char *gqa_last_error_string(void);
+
+/* ABI version of this header: major * 100 + minor. */
+GQA_API int gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GQA_H */

@@ -1,0 +1,177 @@
+"""Grouped-query attention (GQA) on NVIDIA B200: Python binding of libgqa.so.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/gqa.h``.  Tensors are torch
+CUDA tensors (torch provides device memory and streams); there is no CPU or
+library fallback, and importing this module fails loudly when the compiled
+library is missing.
+
+Calls (same names as the C ABI, without the ``gqa_`` prefix):
+
+* :func:`decode` -- one decode step over a [B, G, T_cap, d_h] KV cache.
+* :func:`prefill_causal` -- causal attention over a whole prompt.
+* :func:`meanpool_kv` -- averaging-init of G K/V heads from H MHA heads.
+* :func:`kv_cache_bytes` -- KV-cache bytes per token, 2*G*d_h*L*elem_bytes.
+* :func:`get_status` -- device-side status of earlier calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = ["decode", "decode_workspace_bytes", "prefill_causal", "meanpool_kv",
+           "kv_cache_bytes", "get_status", "GQAError", "LIB_PATH", "lib"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqa.so")
+
+GQA_F32, GQA_BF16 = 0, 1
+_ERRORS = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGN", -4: "CUDA", -5: "WORKSPACE",
+           -6: "TIMEOUT", -7: "SEQLEN"}
+
+# Every symbol include/gqa.h declares.
+EXPORTS = ("gqa_kv_cache_bytes", "gqa_decode_workspace_bytes", "gqa_decode",
+           "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_status",
+           "gqa_last_error_string", "gqa_version")
+
+
+class GQAError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__("GQA_ERR_%s (%d): %s" % (_ERRORS.get(code, "?"), code, msg))
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libgqa.so is not built (expected at %s); run "
+                          "`python kv_cache_decode_04_b200/build.py`" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.gqa_kv_cache_bytes.argtypes = [i32, i32, i32, i32]
+    L.gqa_kv_cache_bytes.restype = ctypes.c_uint64
+    L.gqa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.gqa_decode_workspace_bytes.restype = sz
+    L.gqa_decode.argtypes = [vp, vp, vp, vp, f32, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]
+    L.gqa_decode.restype = i32
+    L.gqa_prefill_causal.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, vp]
+    L.gqa_prefill_causal.restype = i32
+    L.gqa_meanpool_kv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
+    L.gqa_meanpool_kv.restype = i32
+    L.gqa_get_status.argtypes = [vp]
+    L.gqa_get_status.restype = i32
+    L.gqa_last_error_string.argtypes = []
+    L.gqa_last_error_string.restype = ctypes.c_char_p
+    L.gqa_version.restype = i32
+    return L
+
+
+lib = _load()
+
+
+def _check(rc):
+    if rc != 0:
+        raise GQAError(rc, lib.gqa_last_error_string().decode())
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return GQA_BF16
+    if t.dtype == torch.float32:
+        return GQA_F32
+    raise TypeError("GQA tensors must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _dev(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t.data_ptr()
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def kv_cache_bytes(G: int, d_h: int, L: int, elem_bytes: int) -> int:
+    """KV-cache bytes per token: 2 * G * d_h * L * elem_bytes."""
+    return int(lib.gqa_kv_cache_bytes(G, d_h, L, elem_bytes))
+
+
+def decode_workspace_bytes(B, H, G, d_h, T_cap, dtype=torch.bfloat16) -> int:
+    code = GQA_BF16 if dtype == torch.bfloat16 else GQA_F32
+    n = int(lib.gqa_decode_workspace_bytes(B, H, G, d_h, T_cap, code))
+    if n == 0:
+        raise GQAError(-1, "invalid decode shape or device: " + lib.gqa_last_error_string().decode())
+    return n
+
+
+def decode(q, k_cache, v_cache, seqlens, scale=None, out=None, workspace=None, stream=None):
+    """GQA decode: out[b,i] = softmax(scale q[b,i].K[b,g]^T over t < seqlens[b]) V[b,g].
+
+    q [B,H,d_h]; k_cache, v_cache [B,G,T_cap,d_h]; seqlens [B] int32 (device);
+    scale defaults to 1/sqrt(d_h).  Returns ``out`` [B,H,d_h].
+    """
+    B, H, d_h = q.shape
+    Bk, G, T_cap, dk = k_cache.shape
+    if Bk != B or dk != d_h or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between q, k_cache and v_cache")
+    if q.dtype != k_cache.dtype or q.dtype != v_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share a dtype")
+    if seqlens.dtype != torch.int32 or seqlens.numel() != B:
+        raise ValueError("seqlens must be int32 [B]")
+    code = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_h)
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_bytes(B, H, G, d_h, T_cap, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = lib.gqa_decode(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                        _dev(seqlens, "seqlens"), float(scale), _dev(out, "out"), B, H, G, d_h,
+                        T_cap, code, _dev(workspace, "workspace"), workspace.numel(),
+                        _stream(stream))
+    _check(rc)
+    return out
+
+
+def prefill_causal(q, k, v, scale=None, out=None, stream=None):
+    """Causal GQA prefill: q [B,S,H,d_h], k/v [B,S,G,d_h] bf16 -> out [B,S,H,d_h]."""
+    B, S, H, d_h = q.shape
+    G = k.shape[2]
+    if tuple(k.shape) != (B, S, G, d_h) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("shape mismatch between q, k and v")
+    code = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_h)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib.gqa_prefill_causal(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
+                                B, S, H, G, d_h, float(scale), code, _stream(stream))
+    _check(rc)
+    return out
+
+
+def meanpool_kv(wk, wv, G, out_k=None, out_v=None, stream=None):
+    """Averaging init: [H,d_h,d] MHA K/V projections -> [G,d_h,d] group means."""
+    H, d_h, d = wk.shape
+    if tuple(wv.shape) != tuple(wk.shape) or wk.dtype != wv.dtype:
+        raise ValueError("WK and WV must have the same shape and dtype")
+    code = _dtype_code(wk)
+    if out_k is None:
+        out_k = torch.empty((G, d_h, d), dtype=wk.dtype, device=wk.device)
+    if out_v is None:
+        out_v = torch.empty((G, d_h, d), dtype=wk.dtype, device=wk.device)
+    rc = lib.gqa_meanpool_kv(_dev(wk, "WK"), _dev(wv, "WV"), _dev(out_k, "WK_out"),
+                             _dev(out_v, "WV_out"), H, int(G), d_h, d, code, _stream(stream))
+    _check(rc)
+    return out_k, out_v
+
+
+def get_status(stream=None):
+    """Synchronise the stream and raise GQAError if a kernel flagged a device condition."""
+    _check(lib.gqa_get_status(_stream(stream)))

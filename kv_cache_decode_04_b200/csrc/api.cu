@@ -1,0 +1,329 @@
+// api.cu -- the extern "C" boundary of libgqa.so (declared in include/gqa.h).
+//
+// Host-side only: argument validation, TMA tensor-map encoding, the device
+// status word, and the kernel launches.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "gqa.h"
+#include "internal.h"
+
+namespace gqa {
+__device__ unsigned g_status_word;  // bits: see common.cuh
+}
+
+namespace {
+
+thread_local char t_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_err, sizeof t_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int fail_cuda(cudaError_t e, const char *what) {
+    cudaGetLastError();  // clear a non-sticky error
+    return fail(GQA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool misaligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int num_sms = 0;
+    unsigned *status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Per-device facts, set up once per device with that device current.
+int device_info(DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(GQA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        cudaDeviceProp prop;
+        e = cudaGetDeviceProperties(&prop, dev);
+        if (e != cudaSuccess) return fail_cuda(e, "cudaGetDeviceProperties");
+        if (prop.major != 10)
+            return fail(GQA_ERR_UNSUPPORTED, "libgqa is built for sm_100a; device %d is sm_%d%d", dev,
+                        prop.major, prop.minor);
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, gqa::g_status_word);
+        if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(status word)");
+        d.num_sms = prop.multiProcessorCount;
+        d.status = static_cast<unsigned *>(p);
+        d.ready = true;
+    }
+    *out = &d;
+    return GQA_OK;
+}
+
+uint64_t wait_timeout_ns() {
+    static uint64_t v = [] {
+        const char *s = getenv("GQA_WAIT_TIMEOUT_NS");
+        const unsigned long long x = s ? strtoull(s, nullptr, 10) : 0ull;
+        return x ? (uint64_t)x : (uint64_t)2000000000ull;  // 2 s
+    }();
+    return v;
+}
+
+int forced_splits() {
+    const char *s = getenv("GQA_DECODE_CTAS");
+    return s ? atoi(s) : 0;
+}
+
+// ------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encoder(EncodeTiledFn *fn) {
+    static EncodeTiledFn cached = nullptr;
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    if (!cached) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+    *fn = cached;
+    return GQA_OK;
+}
+
+// bf16 tensor of `rank` dims (innermost first), 128-byte swizzled boxes.
+int make_tmap_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                   const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+    EncodeTiledFn enc;
+    int rc = get_encoder(&enc);
+    if (rc) return rc;
+    cuuint32_t elem[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims,
+                     strides_bytes, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return GQA_OK;
+}
+
+int check_dims(int B, int H, int G, int d_h) {
+    if (B <= 0 || H <= 0 || G <= 0 || d_h <= 0)
+        return fail(GQA_ERR_INVALID, "dimensions must be positive (B=%d H=%d G=%d d_h=%d)", B, H, G, d_h);
+    if (H % G != 0) return fail(GQA_ERR_INVALID, "G=%d must divide H=%d", G, H);
+    return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gqa_version(void) { return 100; }
+
+const char *gqa_last_error_string(void) { return t_err; }
+
+uint64_t gqa_kv_cache_bytes(int G, int d_h, int L, int elem_bytes) {
+    if (G <= 0 || d_h <= 0 || L <= 0 || elem_bytes <= 0) return 0;
+    return 2ull * (uint64_t)G * (uint64_t)d_h * (uint64_t)L * (uint64_t)elem_bytes;
+}
+
+size_t gqa_decode_workspace_bytes(int B, int H, int G, int d_h, int T_cap, gqa_dtype dt) {
+    if (check_dims(B, H, G, d_h) || T_cap <= 0) return 0;
+    if (dt != GQA_BF16 && dt != GQA_F32) return 0;
+    DeviceInfo *d = nullptr;
+    if (device_info(&d)) return 0;
+    return gqa::decode_layout(B, H, G, d_h, T_cap, dt, d->num_sms, forced_splits()).total;
+}
+
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+               float scale, void *out, int B, int H, int G, int d_h, int T_cap, gqa_dtype dt,
+               void *workspace, size_t workspace_bytes, gqa_stream_t stream) {
+    t_err[0] = 0;
+    int rc = check_dims(B, H, G, d_h);
+    if (rc) return rc;
+    if (T_cap <= 0) return fail(GQA_ERR_INVALID, "T_cap must be positive");
+    if (!q || !k_cache || !v_cache || !seqlens || !out) return fail(GQA_ERR_INVALID, "null tensor pointer");
+    if (!std::isfinite(scale)) return fail(GQA_ERR_INVALID, "scale must be finite");
+    if (dt != GQA_BF16 && dt != GQA_F32) return fail(GQA_ERR_UNSUPPORTED, "dtype %d", (int)dt);
+    if (d_h != 64 && d_h != 128) return fail(GQA_ERR_UNSUPPORTED, "d_h=%d (built: 64, 128)", d_h);
+    const int r = H / G;
+    if (dt == GQA_BF16 && r > 64) return fail(GQA_ERR_UNSUPPORTED, "bf16 decode needs H/G <= 64 (got %d)", r);
+    if ((long long)B * G * T_cap >= (1ll << 31))
+        return fail(GQA_ERR_UNSUPPORTED, "B*G*T_cap must be below 2^31 rows");
+    if (B > 8192) return fail(GQA_ERR_UNSUPPORTED, "B=%d above 8192", B);
+    if (misaligned(q, 16) || misaligned(k_cache, 16) || misaligned(v_cache, 16) || misaligned(out, 16) ||
+        misaligned(seqlens, 4))
+        return fail(GQA_ERR_ALIGN, "q, k_cache, v_cache and out must be 16-byte aligned");
+    if (gqa::decode_smem_bytes(B, H, G, d_h, dt) > 227u * 1024u)
+        return fail(GQA_ERR_UNSUPPORTED, "shape needs more shared memory than a CTA has (B or H/G too large)");
+    DeviceInfo *d = nullptr;
+    rc = device_info(&d);
+    if (rc) return rc;
+    const gqa::DecodeLayout L = gqa::decode_layout(B, H, G, d_h, T_cap, dt, d->num_sms, forced_splits());
+    if (!workspace || workspace_bytes < L.total)
+        return fail(GQA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (misaligned(workspace, 256)) return fail(GQA_ERR_ALIGN, "workspace must be 256-byte aligned");
+
+    CUtensorMap tmk, tmv;
+    memset(&tmk, 0, sizeof tmk);
+    memset(&tmv, 0, sizeof tmv);
+    if (dt == GQA_BF16) {
+        const cuuint64_t dims[2] = {(cuuint64_t)d_h, (cuuint64_t)B * G * T_cap};
+        const cuuint64_t strides[1] = {(cuuint64_t)d_h * 2};
+        const cuuint32_t box[2] = {64, 64};
+        rc = make_tmap_bf16(&tmk, k_cache, 2, dims, strides, box);
+        if (rc) return rc;
+        rc = make_tmap_bf16(&tmv, v_cache, 2, dims, strides, box);
+        if (rc) return rc;
+    }
+    gqa::DecodeArgs a = {};
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.seqlens = seqlens;
+    a.out = out;
+    a.scale = scale;
+    a.B = B;
+    a.H = H;
+    a.G = G;
+    a.d_h = d_h;
+    a.T_cap = T_cap;
+    a.dtype = dt;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    a.status = d->status;
+    a.timeout_ns = wait_timeout_ns();
+    a.num_sms = d->num_sms;
+    a.force_ctas = forced_splits();
+    cudaError_t e = gqa::launch_decode(a, &tmk, &tmv, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "decode launch");
+    return GQA_OK;
+}
+
+int gqa_prefill_causal(const void *q, const void *k, const void *v, void *out, int B, int S, int H,
+                       int G, int d_h, float scale, gqa_dtype dt, gqa_stream_t stream) {
+    t_err[0] = 0;
+    int rc = check_dims(B, H, G, d_h);
+    if (rc) return rc;
+    if (S <= 0) return fail(GQA_ERR_INVALID, "S must be positive");
+    if (!q || !k || !v || !out) return fail(GQA_ERR_INVALID, "null tensor pointer");
+    if (!std::isfinite(scale)) return fail(GQA_ERR_INVALID, "scale must be finite");
+    if (dt != GQA_BF16) return fail(GQA_ERR_UNSUPPORTED, "prefill supports bf16 only");
+    if (d_h != 128) return fail(GQA_ERR_UNSUPPORTED, "prefill supports d_h=128 only (got %d)", d_h);
+    if ((H / G) % 2 != 0) return fail(GQA_ERR_UNSUPPORTED, "prefill needs an even H/G (got %d)", H / G);
+    if ((long long)B * S * H >= (1ll << 31)) return fail(GQA_ERR_UNSUPPORTED, "B*S*H must be below 2^31");
+    if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(out, 16))
+        return fail(GQA_ERR_ALIGN, "q, k, v and out must be 16-byte aligned");
+    DeviceInfo *d = nullptr;
+    rc = device_info(&d);
+    if (rc) return rc;
+    // 4-D views (innermost first): q [d_h, H, S, B], k/v [d_h, G, S, B].  Boxes of
+    // [64 dims x 1 head x 128 positions x 1 sequence]; positions past S read as zero.
+    CUtensorMap tmq, tmk, tmv;
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)d_h, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+        const cuuint64_t strides[3] = {(cuuint64_t)d_h * 2, (cuuint64_t)H * d_h * 2,
+                                       (cuuint64_t)S * H * d_h * 2};
+        const cuuint32_t box[4] = {64, 1, 128, 1};
+        rc = make_tmap_bf16(&tmq, q, 4, dims, strides, box);
+        if (rc) return rc;
+    }
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)d_h, (cuuint64_t)G, (cuuint64_t)S, (cuuint64_t)B};
+        const cuuint64_t strides[3] = {(cuuint64_t)d_h * 2, (cuuint64_t)G * d_h * 2,
+                                       (cuuint64_t)S * G * d_h * 2};
+        const cuuint32_t box[4] = {64, 1, 128, 1};
+        rc = make_tmap_bf16(&tmk, k, 4, dims, strides, box);
+        if (rc) return rc;
+        rc = make_tmap_bf16(&tmv, v, 4, dims, strides, box);
+        if (rc) return rc;
+    }
+    gqa::PrefillArgs a = {};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.out = out;
+    a.scale = scale;
+    a.B = B;
+    a.S = S;
+    a.H = H;
+    a.G = G;
+    a.d_h = d_h;
+    a.status = d->status;
+    a.timeout_ns = wait_timeout_ns();
+    a.num_sms = d->num_sms;
+    cudaError_t e = gqa::launch_prefill(a, &tmq, &tmk, &tmv, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "prefill launch");
+    return GQA_OK;
+}
+
+int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *WV_out, int H, int G, int d_h,
+                    int d, gqa_dtype dt, gqa_stream_t stream) {
+    t_err[0] = 0;
+    if (H <= 0 || G <= 0 || d_h <= 0 || d <= 0)
+        return fail(GQA_ERR_INVALID, "dimensions must be positive (H=%d G=%d d_h=%d d=%d)", H, G, d_h, d);
+    if (H % G != 0) return fail(GQA_ERR_INVALID, "G=%d must divide H=%d", G, H);
+    if (!WK || !WV || !WK_out || !WV_out) return fail(GQA_ERR_INVALID, "null tensor pointer");
+    if (dt != GQA_BF16 && dt != GQA_F32) return fail(GQA_ERR_UNSUPPORTED, "dtype %d", (int)dt);
+    const size_t esz = dt == GQA_BF16 ? 2 : 4;
+    if (misaligned(WK, esz) || misaligned(WV, esz) || misaligned(WK_out, esz) || misaligned(WV_out, esz))
+        return fail(GQA_ERR_ALIGN, "tensors must be aligned to their element size");
+    const long long n = (long long)d_h * d;
+    // the outputs must not overlap the inputs
+    const char *ik = static_cast<const char *>(WK), *iv = static_cast<const char *>(WV);
+    const char *okp = static_cast<const char *>(WK_out), *ovp = static_cast<const char *>(WV_out);
+    const long long in_b = (long long)H * n * esz, out_b = (long long)G * n * esz;
+    auto overlap = [](const char *a, long long na, const char *b, long long nb) {
+        return a < b + nb && b < a + na;
+    };
+    if (overlap(ik, in_b, okp, out_b) || overlap(ik, in_b, ovp, out_b) || overlap(iv, in_b, okp, out_b) ||
+        overlap(iv, in_b, ovp, out_b) || overlap(okp, out_b, ovp, out_b))
+        return fail(GQA_ERR_INVALID, "output tensors overlap an input or each other");
+    DeviceInfo *d_ = nullptr;
+    int rc = device_info(&d_);
+    if (rc) return rc;
+    cudaError_t e = gqa::launch_meanpool(WK, WV, WK_out, WV_out, H, G, n, dt, d_->num_sms,
+                                         reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "meanpool launch");
+    return GQA_OK;
+}
+
+int gqa_get_status(gqa_stream_t stream) {
+    t_err[0] = 0;
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "cudaStreamSynchronize");
+    DeviceInfo *d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    unsigned word = 0;
+    e = cudaMemcpy(&word, d->status, sizeof word, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail_cuda(e, "reading the status word");
+    if (word) {
+        const unsigned zero = 0;
+        e = cudaMemcpy(d->status, &zero, sizeof zero, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return fail_cuda(e, "clearing the status word");
+    }
+    if (word & 2u) return fail(GQA_ERR_TIMEOUT, "a device-side wait ran out of time");
+    if (word & 1u) return fail(GQA_ERR_SEQLEN, "a seqlens entry was outside [0, T_cap] (clamped)");
+    return GQA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,706 @@
+// decode.cu -- GQA decode over a [B, G, T_cap, d_h] KV cache (sm_100a).
+//
+// What is computed ("Grouped-Query Attention", llm-arch-kb, sections 1-3):
+// for every sequence b and query head i, with g = i / (H/G),
+//     out[b,i] = sum_{t < T_b} softmax_t(scale * q[b,i] . K[b,g,t]) V[b,g,t].
+// Every cached key and value is read once per decode step; the H/G query
+// heads of a group share the one K/V head, so a K/V tile staged in shared
+// memory serves all of them.
+//
+// How (split-KV, two kernels):
+//   1. decode_split_*: the cache tiles of all (b, g) segments are laid end to
+//      end and cut into gridDim.x equal shares; CTA c takes share c.  A share
+//      may cover the tail of one segment and the head of the next.  For each
+//      piece (the part of one segment inside one share) the CTA emits a
+//      partial record (running max m, sum l, unnormalised output o) per query
+//      head, at record index c + segment (distinct for all pieces: two pieces
+//      with equal c + segment would need an earlier CTA to hold a later
+//      segment).
+//   2. decode_combine: for each (b, i) merges the records of its segment:
+//      M = max m_c, L = sum 2^(m_c - M) l_c, out = sum 2^(m_c - M) o_c / L.
+//   Softmax runs in the base-2 domain on scores pre-multiplied by
+//   scale*log2(e), which leaves the result unchanged.
+//
+// bf16 path: a producer warp streams [64 x d_h] K and V tiles with TMA
+// (128-byte swizzle) through a 4-stage mbarrier ring; four consumer warps run
+// warp-level bf16 tensor-core MMAs (scores, then P.V with P rounded to bf16)
+// and an fp32 online softmax; query rows are padded to 16 per MMA tile.
+// fp32 path: CUDA-core fp32 arithmetic throughout (no TF32).
+#include "common.cuh"
+#include "gqa.h"
+#include "internal.h"
+
+namespace gqa {
+
+namespace {
+
+constexpr int kTile = 64;       // tokens per K/V tile, bf16 path
+constexpr int kTileF32 = 32;    // tokens per tile, fp32 path
+constexpr int kStages = 4;      // TMA ring depth
+constexpr int kCWarps = 4;      // consumer warps
+constexpr int kThreads = (kCWarps + 1) * 32;
+constexpr int kHalfBytes = kTile * 128;  // one [64 tokens x 64 dims] bf16 box
+constexpr int kThreadsF32 = 128;
+
+struct DecodeParams {
+    const void *q;
+    const int32_t *seqlens;
+    void *out;
+    int *ws_cu;     // [B+1] tile prefix, written by CTA 0 of the split kernel
+    float2 *ws_ml;  // [n_rec * r]: (max in log2 units, sum)
+    float *ws_o;    // [n_rec * r * d_h]: unnormalised outputs
+    const float *k32, *v32;  // fp32 path only
+    unsigned *status;
+    float scale_log2;
+    int B, H, G, r, T_cap;
+    unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ int clamp_len(int T, int T_cap) {
+    return T < 0 ? 0 : (T > T_cap ? T_cap : T);
+}
+
+// cu[b] = G * sum_{b' < b} ceil(T_b' / TILE), T clamped to [0, T_cap];
+// cu[B] = total tiles W.  Every thread of the block must call it.
+template <int TILE>
+__device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, bool report) {
+    const int nt = blockDim.x, tid = threadIdx.x;
+    const int chunk = (p.B + nt - 1) / nt;
+    const int b0 = min(p.B, tid * chunk), b1 = min(p.B, b0 + chunk);
+    int local = 0;
+    bool bad = false;
+    for (int b = b0; b < b1; ++b) {
+        const int T = p.seqlens[b];
+        bad |= (T < 0 || T > p.T_cap);
+        local += (clamp_len(T, p.T_cap) + TILE - 1) / TILE;
+    }
+    if (bad && report) set_status(p.status, STATUS_SEQLEN);
+    scratch[tid] = local;
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int i = 0; i < nt; ++i) {
+            const int v = scratch[i];
+            scratch[i] = run;
+            run += v;
+        }
+        cu[p.B] = run * p.G;
+    }
+    __syncthreads();
+    int run = scratch[tid];
+    for (int b = b0; b < b1; ++b) {
+        cu[b] = run * p.G;
+        run += (clamp_len(p.seqlens[b], p.T_cap) + TILE - 1) / TILE;
+    }
+    __syncthreads();
+    return cu[p.B];
+}
+
+// Position in the tile line: sequence b, KV head g, tile j of the segment,
+// tiles per segment of b.
+struct Cursor {
+    int b, g, j, ntb;
+};
+
+__device__ __forceinline__ void cursor_seek(const int *cu, int B, int G, int u, Cursor &c) {
+    int lo = 0, hi = B - 1;  // largest b with cu[b] <= u (then cu[b] <= u < cu[b+1])
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cu[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    c.b = lo;
+    c.ntb = (cu[lo + 1] - cu[lo]) / G;
+    const int off = u - cu[lo];
+    c.g = off / c.ntb;
+    c.j = off - c.g * c.ntb;
+}
+
+__device__ __forceinline__ void cursor_next(const int *cu, int B, int G, Cursor &c) {
+    if (++c.j < c.ntb) return;
+    c.j = 0;
+    if (++c.g < G) return;
+    c.g = 0;
+    do {
+        ++c.b;
+    } while (c.b < B && cu[c.b + 1] == cu[c.b]);
+    if (c.b < B) c.ntb = (cu[c.b + 1] - cu[c.b]) / G;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16 *p) {
+    return *reinterpret_cast<const uint32_t *>(p);
+}
+
+// Byte offset of (token, dim) inside a stage buffer of [64 x D] bf16 made of
+// D/64 boxes of [64 tokens x 64 dims] with the TMA 128-byte swizzle: the
+// 16-byte chunk index inside a 128-byte row is XORed with (row mod 8).
+__device__ __forceinline__ uint32_t swz(int tok, int dim) {
+    return (uint32_t)((dim >> 6) * kHalfBytes + tok * 128 + ((((dim & 63) >> 3) ^ (tok & 7)) << 4) +
+                      ((dim & 7) << 1));
+}
+
+// ----------------------------------------------------------------- bf16
+
+template <int D, int NMT>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_split_bf16(const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
+    constexpr int HALVES = D / 64;
+    constexpr int KV_BYTES = kTile * D * 2;
+    constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    constexpr int NSL = kCWarps / NMT;  // token slices of a tile
+    constexpr int TPS = kTile / NSL;    // tokens per slice
+    constexpr int ROWF = D + 2;         // reduction row: m, l, o[D]
+    constexpr int RED_FLOATS = NSL > 1 ? NSL * NMT * 16 * ROWF : 0;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint8_t *stages = smem;
+    float *red = reinterpret_cast<float *>(smem + kStages * STAGE_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * STAGE_BYTES + RED_FLOATS * 4);
+    uint64_t *empty = full + kStages;
+    int *abort_flag = reinterpret_cast<int *>(empty + kStages);
+    int *cu = abort_flag + 1;
+    int *scratch = cu + p.B + 1;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kCWarps);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kCWarps && lane == 0) {
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+    }
+    const int W = build_tile_prefix<kTile>(p, cu, scratch, blockIdx.x == 0);
+    if (blockIdx.x == 0)
+        for (int i = tid; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
+    pdl_launch_dependents();
+
+    const long long C = gridDim.x;
+    const int u_begin = (int)((long long)blockIdx.x * W / C);
+    const int u_end = (int)((long long)(blockIdx.x + 1) * W / C);
+    if (u_begin >= u_end) return;
+    volatile int *vabort = abort_flag;
+
+    if (warp == kCWarps) {  // ---------------- producer: TMA ring
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            Cursor c;
+            cursor_seek(cu, p.B, p.G, u_begin, c);
+            for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (*vabort || !mbar_wait(&empty[s], ph ^ 1, p.timeout_ns)) {
+                    set_status(p.status, STATUS_TIMEOUT);
+                    *vabort = 1;
+                    break;
+                }
+                uint8_t *kdst = stages + s * STAGE_BYTES;
+                uint8_t *vdst = kdst + KV_BYTES;
+                mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                const int row = (c.b * p.G + c.g) * p.T_cap + c.j * kTile;
+#pragma unroll
+                for (int h = 0; h < HALVES; ++h) {
+                    tma_load_2d(kdst + h * kHalfBytes, &tmk, &full[s], h * 64, row, pol);
+                    tma_load_2d(vdst + h * kHalfBytes, &tmv, &full[s], h * 64, row, pol);
+                }
+                cursor_next(cu, p.B, p.G, c);
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers
+    const int mt = warp % NMT, sl = warp / NMT;
+    const int g8 = lane >> 2, q4 = lane & 3;
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q);
+
+    uint32_t qa[D / 16][4];
+    float o[D / 8][4];
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    int cur_bg = -1;
+    bool dead = false;  // a wait ran out: keep joining barriers, skip the work
+
+    Cursor c;
+    cursor_seek(cu, p.B, p.G, u_begin, c);
+    for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
+        const int b = c.b, bg = c.b * p.G + c.g;
+        const int t0 = c.j * kTile;
+        const int n_valid = min(kTile, clamp_len(p.seqlens[b], p.T_cap) - t0);
+        if (bg != cur_bg) {  // first tile of a piece: this group's queries
+            cur_bg = bg;
+            const int hl_a = mt * 16 + g8, hl_b = hl_a + 8;
+            const __nv_bfloat16 *qb = qg + ((size_t)b * p.H + (size_t)c.g * p.r) * D;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int col = kk * 16 + 2 * q4;
+                qa[kk][0] = hl_a < p.r ? ld_u32(qb + (size_t)hl_a * D + col) : 0u;
+                qa[kk][1] = hl_b < p.r ? ld_u32(qb + (size_t)hl_b * D + col) : 0u;
+                qa[kk][2] = hl_a < p.r ? ld_u32(qb + (size_t)hl_a * D + col + 8) : 0u;
+                qa[kk][3] = hl_b < p.r ? ld_u32(qb + (size_t)hl_b * D + col + 8) : 0u;
+            }
+#pragma unroll
+            for (int nn = 0; nn < D / 8; ++nn) o[nn][0] = o[nn][1] = o[nn][2] = o[nn][3] = 0.f;
+            m_a = m_b = -INFINITY;
+            l_a = l_b = 0.f;
+        }
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!dead && (*vabort || !mbar_wait(&full[s], ph, p.timeout_ns))) {
+            dead = true;
+            *vabort = 1;
+            set_status(p.status, STATUS_TIMEOUT);
+        }
+        if (!dead) {
+            const uint32_t kbase = smem_u32(stages + s * STAGE_BYTES);
+            const uint32_t vbase = kbase + KV_BYTES;
+#pragma unroll
+            for (int step = 0; step < TPS / 16; ++step) {
+                const int row0 = sl * TPS + step * 16;
+                if (row0 >= n_valid) break;
+                if (row0 + 16 > n_valid) {
+                    // rows past the end of the sequence: zero V so 0 * (garbage) stays 0
+                    for (int idx = lane; idx < 16 * HALVES * 8; idx += 32) {
+                        const int rr = row0 + idx / (HALVES * 8);
+                        const int rem = idx % (HALVES * 8);
+                        if (rr >= n_valid) {
+                            const uint32_t a = vbase + (rem >> 3) * kHalfBytes + rr * 128 + (rem & 7) * 16;
+                            asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(a), "r"(0u)
+                                         : "memory");
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                // S[16 heads x 16 tokens] = q . K^T
+                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                {
+                    const int tok = row0 + ((lane >> 4) << 3) + (lane & 7);
+                    const int dsel = ((lane >> 3) & 1) << 3;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(kbase + swz(tok, kk * 16 + dsel), b0, b1, b2, b3);
+                        mma_16816(sc[0], qa[kk], b0, b1);
+                        mma_16816(sc[1], qa[kk], b2, b3);
+                    }
+                }
+                // scale into the log2 domain, mask tokens past the end
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int tok = row0 + nt * 8 + 2 * q4 + (e & 1);
+                        const float v = sc[nt][e] * p.scale_log2;
+                        sc[nt][e] = tok < n_valid ? v : -INFINITY;
+                    }
+                float mx_a = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+                float mx_b = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+                const float mu_a = mn_a == -INFINITY ? 0.f : mn_a;
+                const float mu_b = mn_b == -INFINITY ? 0.f : mn_b;
+                const float al_a = fast_exp2(m_a - mu_a), al_b = fast_exp2(m_b - mu_b);
+                m_a = mn_a;
+                m_b = mn_b;
+                uint32_t pa[4];
+                float ps_a = 0.f, ps_b = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    pa[2 * nt + 0] = pack_bf16x2(fast_exp2(sc[nt][0] - mu_a), fast_exp2(sc[nt][1] - mu_a));
+                    pa[2 * nt + 1] = pack_bf16x2(fast_exp2(sc[nt][2] - mu_b), fast_exp2(sc[nt][3] - mu_b));
+                    const float2 fa = unpack_bf16x2(pa[2 * nt + 0]);
+                    const float2 fb = unpack_bf16x2(pa[2 * nt + 1]);
+                    ps_a += fa.x + fa.y;
+                    ps_b += fb.x + fb.y;
+                }
+                l_a = l_a * al_a + ps_a;
+                l_b = l_b * al_b + ps_b;
+#pragma unroll
+                for (int nn = 0; nn < D / 8; ++nn) {
+                    o[nn][0] *= al_a;
+                    o[nn][1] *= al_a;
+                    o[nn][2] *= al_b;
+                    o[nn][3] *= al_b;
+                }
+                // O[16 x D] += P[16 x 16] . V[16 x D]
+                {
+                    const int tok = row0 + (((lane >> 3) & 1) << 3) + (lane & 7);
+                    const int dsel = (lane >> 4) << 3;
+#pragma unroll
+                    for (int n2 = 0; n2 < D / 16; ++n2) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(vbase + swz(tok, n2 * 16 + dsel), b0, b1, b2, b3);
+                        mma_16816(o[2 * n2], pa, b0, b1);
+                        mma_16816(o[2 * n2 + 1], pa, b2, b3);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        cursor_next(cu, p.B, p.G, c);
+        const bool piece_end = (u + 1 == u_end) || (c.b * p.G + c.g != bg);
+        if (!piece_end) continue;
+
+        // ---------------- emit this piece's partial record
+        float la = l_a, lb = l_b;
+        la += __shfl_xor_sync(0xffffffffu, la, 1);
+        la += __shfl_xor_sync(0xffffffffu, la, 2);
+        lb += __shfl_xor_sync(0xffffffffu, lb, 1);
+        lb += __shfl_xor_sync(0xffffffffu, lb, 2);
+        const long long rec = (long long)blockIdx.x + bg;
+        if (NSL == 1) {
+            const int hl_a = mt * 16 + g8, hl_b = hl_a + 8;
+            if (!dead && hl_a < p.r) {
+                float *dst = p.ws_o + (rec * p.r + hl_a) * D;
+#pragma unroll
+                for (int nn = 0; nn < D / 8; ++nn)
+                    *reinterpret_cast<float2 *>(dst + nn * 8 + 2 * q4) = make_float2(o[nn][0], o[nn][1]);
+                if (q4 == 0) p.ws_ml[rec * p.r + hl_a] = make_float2(m_a, la);
+            }
+            if (!dead && hl_b < p.r) {
+                float *dst = p.ws_o + (rec * p.r + hl_b) * D;
+#pragma unroll
+                for (int nn = 0; nn < D / 8; ++nn)
+                    *reinterpret_cast<float2 *>(dst + nn * 8 + 2 * q4) = make_float2(o[nn][2], o[nn][3]);
+                if (q4 == 0) p.ws_ml[rec * p.r + hl_b] = make_float2(m_b, lb);
+            }
+        } else {
+            float *ra = red + ((sl * NMT + mt) * 16 + g8) * ROWF;
+            float *rb = ra + 8 * ROWF;
+            if (q4 == 0) {
+                ra[0] = m_a;
+                ra[1] = la;
+                rb[0] = m_b;
+                rb[1] = lb;
+            }
+#pragma unroll
+            for (int nn = 0; nn < D / 8; ++nn) {
+                ra[2 + nn * 8 + 2 * q4] = o[nn][0];
+                ra[3 + nn * 8 + 2 * q4] = o[nn][1];
+                rb[2 + nn * 8 + 2 * q4] = o[nn][2];
+                rb[3 + nn * 8 + 2 * q4] = o[nn][3];
+            }
+            named_bar_sync(1, kCWarps * 32);
+            const int rows = min(p.r, NMT * 16);
+            for (int idx = tid; idx < rows * D; idx += kCWarps * 32) {
+                const int hl = idx / D, col = idx - hl * D;
+                const int mtr = hl >> 4, rr = hl & 15;
+                float M = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < NSL; ++k) M = fmaxf(M, red[((k * NMT + mtr) * 16 + rr) * ROWF]);
+                float acc = 0.f, L = 0.f;
+#pragma unroll
+                for (int k = 0; k < NSL; ++k) {
+                    const float *row = red + ((k * NMT + mtr) * 16 + rr) * ROWF;
+                    const float w = fast_exp2(row[0] - M);
+                    acc += w * row[2 + col];
+                    L += w * row[1];
+                }
+                if (!dead) {
+                    p.ws_o[(rec * p.r + hl) * D + col] = acc;
+                    if (col == 0) p.ws_ml[rec * p.r + hl] = make_float2(M, L);
+                }
+            }
+            named_bar_sync(1, kCWarps * 32);
+        }
+    }
+}
+
+// ----------------------------------------------------------------- fp32
+
+template <int D>
+__global__ void __launch_bounds__(kThreadsF32)
+    decode_split_f32(const DecodeParams p) {
+    constexpr int KS = D + 1;  // padded row stride (bank spread)
+    extern __shared__ float sm32[];
+    float *Ks = sm32;                  // [32][KS]
+    float *Vs = Ks + kTileF32 * KS;    // [32][KS]
+    float *ps = Vs + kTileF32 * KS;    // [4 warps][32]
+    float *qs = ps + 4 * 32;           // [r][D]
+    float *st_o = qs + p.r * D;        // [r][D]
+    float *st_m = st_o + p.r * D;      // [r]
+    float *st_l = st_m + p.r;          // [r]
+    int *cu = reinterpret_cast<int *>(st_l + p.r);
+    int *scratch = cu + p.B + 1;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int W = build_tile_prefix<kTileF32>(p, cu, scratch, blockIdx.x == 0);
+    if (blockIdx.x == 0)
+        for (int i = tid; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
+    pdl_launch_dependents();
+    const long long C = gridDim.x;
+    const int u_begin = (int)((long long)blockIdx.x * W / C);
+    const int u_end = (int)((long long)(blockIdx.x + 1) * W / C);
+    if (u_begin >= u_end) return;
+    const float *qg = static_cast<const float *>(p.q);
+
+    int cur_bg = -1;
+    Cursor c;
+    cursor_seek(cu, p.B, p.G, u_begin, c);
+    for (int u = u_begin; u < u_end; ++u) {
+        const int b = c.b, bg = c.b * p.G + c.g;
+        const int t0 = c.j * kTileF32;
+        const int n_valid = min(kTileF32, clamp_len(p.seqlens[b], p.T_cap) - t0);
+        if (bg != cur_bg) {
+            cur_bg = bg;
+            const float *qb = qg + ((size_t)b * p.H + (size_t)c.g * p.r) * D;
+            for (int i = tid; i < p.r * D; i += blockDim.x) {
+                qs[i] = qb[i];
+                st_o[i] = 0.f;
+            }
+            for (int i = tid; i < p.r; i += blockDim.x) {
+                st_m[i] = -INFINITY;
+                st_l[i] = 0.f;
+            }
+        }
+        const size_t base = ((size_t)bg * p.T_cap + t0) * D;
+        for (int i = tid; i < kTileF32 * D; i += blockDim.x) {
+            const int row = i / D, col = i - row * D;
+            const bool ok = row < n_valid;
+            Ks[row * KS + col] = ok ? p.k32[base + i] : 0.f;
+            Vs[row * KS + col] = ok ? p.v32[base + i] : 0.f;
+        }
+        __syncthreads();
+        for (int hl = warp; hl < p.r; hl += 4) {
+            float s = -INFINITY;
+            if (lane < n_valid) {
+                float acc = 0.f;
+                for (int k = 0; k < D; ++k) acc = fmaf(qs[hl * D + k], Ks[lane * KS + k], acc);
+                s = acc * p.scale_log2;
+            }
+            float mx = s;
+#pragma unroll
+            for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float m_old = st_m[hl];
+            const float m_new = fmaxf(m_old, mx);  // finite: token 0 of a tile is valid
+            const float alpha = fast_exp2(m_old - m_new);
+            const float pr = fast_exp2(s - m_new);
+            float sum = pr;
+#pragma unroll
+            for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            ps[warp * 32 + lane] = pr;
+            __syncwarp();
+            for (int col = lane; col < D; col += 32) {
+                float acc = st_o[hl * D + col] * alpha;
+                for (int t = 0; t < n_valid; ++t) acc = fmaf(ps[warp * 32 + t], Vs[t * KS + col], acc);
+                st_o[hl * D + col] = acc;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                st_m[hl] = m_new;
+                st_l[hl] = st_l[hl] * alpha + sum;
+            }
+            __syncwarp();
+        }
+        __syncthreads();
+        cursor_next(cu, p.B, p.G, c);
+        const bool piece_end = (u + 1 == u_end) || (c.b * p.G + c.g != bg);
+        if (piece_end) {
+            const long long rec = (long long)blockIdx.x + bg;
+            for (int i = tid; i < p.r * D; i += blockDim.x) p.ws_o[rec * p.r * D + i] = st_o[i];
+            for (int i = tid; i < p.r; i += blockDim.x)
+                p.ws_ml[rec * p.r + i] = make_float2(st_m[i], st_l[i]);
+            __syncthreads();
+        }
+    }
+}
+
+// ----------------------------------------------------------------- combine
+
+template <int D, bool BF16_OUT>
+__global__ void __launch_bounds__(128) decode_combine(const DecodeParams p, int C) {
+    pdl_wait_primary();  // the split kernel's records are complete and visible
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 4 + warp;  // b*H + h
+    if (row >= (long long)p.B * p.H) return;
+    const int b = (int)(row / p.H), h = (int)(row % p.H);
+    const int g = h / p.r, hl = h - g * p.r;
+    const int bg = b * p.G + g;
+    constexpr int PER = D / 32;
+    float acc[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc[k] = 0.f;
+    const int *cu = p.ws_cu;
+    const int ntb = (cu[b + 1] - cu[b]) / p.G;
+    if (ntb > 0) {
+        const long long W = cu[p.B];
+        const long long s0 = cu[b] + (long long)g * ntb, s1 = s0 + ntb;
+        const int c_lo = (int)(((s0 + 1) * C - 1) / W);
+        const int c_hi = (int)((s1 * C - 1) / W);
+        // CTAs whose share is empty (more CTAs than tiles) wrote no record
+        auto empty_share = [&](int c) { return (long long)c * W / C == (long long)(c + 1) * W / C; };
+        float M = -INFINITY;
+        for (int c = c_lo; c <= c_hi; ++c)
+            if (!empty_share(c)) M = fmaxf(M, p.ws_ml[((long long)c + bg) * p.r + hl].x);
+        float L = 0.f;
+        for (int c = c_lo; c <= c_hi; ++c) {
+            if (empty_share(c)) continue;
+            const long long rec = (long long)c + bg;
+            const float2 ml = p.ws_ml[rec * p.r + hl];
+            const float w = fast_exp2(ml.x - M);
+            L += w * ml.y;
+            const float *src = p.ws_o + (rec * p.r + hl) * D + lane * PER;
+            if constexpr (PER == 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(src);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+                acc[2] += w * v.z;
+                acc[3] += w * v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2 *>(src);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+            }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) acc[k] *= inv;
+    }
+    if constexpr (BF16_OUT) {
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + row * D + lane * PER;
+        if constexpr (PER == 4)
+            *reinterpret_cast<uint2 *>(dst) =
+                make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+        else
+            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0], acc[1]);
+    } else {
+        float *dst = static_cast<float *>(p.out) + row * D + lane * PER;
+        if constexpr (PER == 4)
+            *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        else
+            *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1]);
+    }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int bf16_nmt(int r) { return r <= 16 ? 1 : (r <= 32 ? 2 : 4); }
+
+size_t smem_bf16(int D, int nmt, int B) {
+    const int nsl = kCWarps / nmt;
+    const size_t red = nsl > 1 ? (size_t)nsl * nmt * 16 * (D + 2) * 4 : 0;
+    return 1024 + (size_t)kStages * 2 * kTile * D * 2 + red + 2 * kStages * 8 + 4 +
+           (size_t)(B + 1) * 4 + kThreads * 4;
+}
+
+size_t smem_f32(int D, int r, int B) {
+    return ((size_t)2 * kTileF32 * (D + 1) + 4 * 32 + 2 * (size_t)r * D + 2 * r) * 4 +
+           (size_t)(B + 1) * 4 + kThreadsF32 * 4;
+}
+
+template <int D, int NMT>
+cudaError_t run_bf16(const DecodeParams &p, const CUtensorMap *tmk, const CUtensorMap *tmv,
+                     int ctas, cudaStream_t st) {
+    const size_t smem = smem_bf16(D, NMT, p.B);
+    auto kern = decode_split_bf16<D, NMT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, kThreads, smem, st>>>(*tmk, *tmv, p);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t run_f32(const DecodeParams &p, int ctas, cudaStream_t st) {
+    const size_t smem = smem_f32(D, p.r, p.B);
+    auto kern = decode_split_f32<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, kThreadsF32, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <int D, bool BF16_OUT>
+cudaError_t run_combine(const DecodeParams &p, int ctas, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(((long long)p.B * p.H + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT>, p, ctas);
+}
+
+}  // namespace
+
+DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, int num_sms,
+                           int force_ctas) {
+    DecodeLayout L = {};
+    const int r = H / G;
+    const int tile = dtype == GQA_BF16 ? kTile : kTileF32;
+    const long long max_tiles = (long long)B * G * ((T_cap + tile - 1) / tile);
+    long long ctas = force_ctas > 0 ? force_ctas : (long long)num_sms;
+    if (ctas > max_tiles) ctas = max_tiles;
+    if (ctas < 1) ctas = 1;
+    L.ctas = (int)ctas;
+    L.n_rec = ctas + (long long)B * G;
+    L.off_cu = 0;
+    L.off_ml = align256((size_t)(B + 1) * 4);
+    L.off_o = L.off_ml + align256((size_t)L.n_rec * r * sizeof(float2));
+    L.total = L.off_o + align256((size_t)L.n_rec * r * d_h * sizeof(float));
+    return L;
+}
+
+size_t decode_smem_bytes(int B, int H, int G, int d_h, int dtype) {
+    const int r = H / G;
+    return dtype == GQA_BF16 ? smem_bf16(d_h, bf16_nmt(r), B) : smem_f32(d_h, r, B);
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUtensorMap *tmv,
+                          cudaStream_t st) {
+    const DecodeLayout L = decode_layout(a.B, a.H, a.G, a.d_h, a.T_cap, a.dtype, a.num_sms, a.force_ctas);
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    DecodeParams p = {};
+    p.q = a.q;
+    p.seqlens = a.seqlens;
+    p.out = a.out;
+    p.ws_cu = reinterpret_cast<int *>(ws + L.off_cu);
+    p.ws_ml = reinterpret_cast<float2 *>(ws + L.off_ml);
+    p.ws_o = reinterpret_cast<float *>(ws + L.off_o);
+    p.k32 = static_cast<const float *>(a.k_cache);
+    p.v32 = static_cast<const float *>(a.v_cache);
+    p.status = a.status;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.B = a.B;
+    p.H = a.H;
+    p.G = a.G;
+    p.r = a.H / a.G;
+    p.T_cap = a.T_cap;
+    p.timeout_ns = a.timeout_ns;
+    cudaError_t e;
+    if (a.dtype == GQA_BF16) {
+        const int nmt = bf16_nmt(p.r);
+        if (a.d_h == 128)
+            e = nmt == 1 ? run_bf16<128, 1>(p, tmk, tmv, L.ctas, st)
+              : nmt == 2 ? run_bf16<128, 2>(p, tmk, tmv, L.ctas, st)
+                         : run_bf16<128, 4>(p, tmk, tmv, L.ctas, st);
+        else
+            e = nmt == 1 ? run_bf16<64, 1>(p, tmk, tmv, L.ctas, st)
+              : nmt == 2 ? run_bf16<64, 2>(p, tmk, tmv, L.ctas, st)
+                         : run_bf16<64, 4>(p, tmk, tmv, L.ctas, st);
+        if (e != cudaSuccess) return e;
+        return a.d_h == 128 ? run_combine<128, true>(p, L.ctas, st) : run_combine<64, true>(p, L.ctas, st);
+    }
+    e = a.d_h == 128 ? run_f32<128>(p, L.ctas, st) : run_f32<64>(p, L.ctas, st);
+    if (e != cudaSuccess) return e;
+    return a.d_h == 128 ? run_combine<128, false>(p, L.ctas, st) : run_combine<64, false>(p, L.ctas, st);
+}
+
+}  // namespace gqa

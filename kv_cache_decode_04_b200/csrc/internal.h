@@ -1,0 +1,61 @@
+// internal.h -- launchers shared between the C-ABI layer and the kernel files.
+// Not installed; the public interface is include/gqa.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gqa {
+
+// Split-KV decode: one pass over equal shares of the cache tiles, then a
+// combine pass.  Partial records live in the caller's workspace.
+struct DecodeArgs {
+    const void *q;
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *seqlens;
+    void *out;
+    float scale;
+    int B, H, G, d_h, T_cap;
+    int dtype;  // gqa_dtype
+    void *workspace;
+    size_t workspace_bytes;
+    unsigned *status;
+    uint64_t timeout_ns;
+    int num_sms;
+    int force_ctas;  // >0: use this many split CTAs (tests of the split logic)
+};
+
+// Workspace layout, all offsets 256-byte aligned.
+struct DecodeLayout {
+    int ctas;          // split CTAs of the first kernel
+    long long n_rec;   // partial records: ctas + B*G
+    size_t off_cu, off_ml, off_o, total;
+};
+
+DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, int num_sms,
+                           int force_ctas);
+size_t decode_smem_bytes(int B, int H, int G, int d_h, int dtype);
+cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUtensorMap *tmv,
+                          cudaStream_t stream);
+
+// Prefill (tcgen05).  Tensor maps over q, k, v built by the caller.
+struct PrefillArgs {
+    const void *q, *k, *v;
+    void *out;
+    float scale;
+    int B, S, H, G, d_h;
+    unsigned *status;
+    uint64_t timeout_ns;
+    int num_sms;
+};
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const CUtensorMap *tmk,
+                           const CUtensorMap *tmv, cudaStream_t stream);
+
+// Mean-pool init.
+cudaError_t launch_meanpool(const void *wk, const void *wv, void *ok, void *ov, int H, int G,
+                            long long n, int dtype, int num_sms, cudaStream_t stream);
+
+}  // namespace gqa

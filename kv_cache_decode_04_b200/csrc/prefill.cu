@@ -1,0 +1,372 @@
+// prefill.cu -- causal GQA prefill on the 5th-generation tensor cores (sm_100a).
+//
+// What is computed ("Grouped-Query Attention", llm-arch-kb, section 3
+// "Reference implementation"): for each sequence b, position s and query head
+// i with g = i / (H/G),
+//     out[b,s,i] = sum_{t <= s} softmax_t(scale * q[b,s,i] . k[b,t,g]) v[b,t,g].
+// GQA does not reduce the flops of this step (each query head still scores
+// every key), so QK^T and PV are dense tensor-core contractions here.
+//
+// One CTA = 128 query positions x 2 query heads of the same group: both heads
+// read the same K/V tiles, which each load therefore serves twice.
+//   warp 8      TMA producer: Q tiles once, then [128 x 128] K and V tiles of
+//               the group through 2-stage rings (128-byte swizzle).
+//   warp 9      allocates 512 tensor-memory columns; one lane issues every
+//               tcgen05.mma:  S_h = Q_h K_j^T  (fp32 in TMEM, 128 cols each)
+//                             O_h += P_h V_j   (P read from TMEM, fp32 O in TMEM)
+//   warps 0-3   softmax + epilogue for head 0 (one thread per query row =
+//   warps 4-7   one TMEM lane), head 1.  While one group runs its softmax the
+//               tensor core works on the other head's MMAs.
+// TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,384) O0, [384,512) O1.
+// P (bf16) overwrites the first 64 columns of its S block after S is read.
+// Online softmax in the base-2 domain; the running max is only moved (and O
+// rescaled in TMEM) when it grows by more than 8, so p <= 2^8: the result is
+// the same because numerator and denominator use the same stale maximum.
+// Only KV tiles j <= query tile are visited; the diagonal tile is masked
+// (key > query -> -inf).
+#include "common.cuh"
+#include "gqa.h"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace gqa {
+
+namespace {
+
+constexpr int kBM = 128;                 // query rows per tile
+constexpr int kBN = 128;                 // keys per KV tile
+constexpr int kHalf = 128 * 64 * 2;      // one [128 rows x 64 bf16] swizzled box
+constexpr int kTile = 2 * kHalf;         // [128 x 128] bf16
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kOffQ = 0;                 // Q0, Q1
+constexpr int kOffK = 2 * kTile;         // K stages 0, 1
+constexpr int kOffV = 4 * kTile;         // V stages 0, 1
+constexpr int kOffBar = 6 * kTile;
+constexpr size_t kSmemBytes = 1024 + kOffBar + 256;
+
+struct PrefillParams {
+    void *out;
+    unsigned *status;
+    float scale_log2;
+    int B, S, H, G, r, n_qt;
+    unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, uint64_t *bar, int x, int y,
+                                            int z, int w, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w),
+        "l"(policy)
+        : "memory");
+}
+
+// Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64_t limit) {
+    const bool ok = mbar_wait(bar, parity, limit);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_causal_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                          const __grid_constant__ CUtensorMap tmv, const PrefillParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
+    uint64_t *bar_q = bars + 0;
+    uint64_t *k_full = bars + 1;   // [2]
+    uint64_t *k_empty = bars + 3;  // [2]
+    uint64_t *v_full = bars + 5;   // [2]
+    uint64_t *v_empty = bars + 7;  // [2]
+    uint64_t *s_full = bars + 9;   // [2] one per head
+    uint64_t *p_ready = bars + 11; // [2]
+    uint64_t *o_done = bars + 13;
+    uint64_t *drain = bars + 14;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    volatile int *vabort = abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // work unit: heaviest query tiles (most KV tiles) first
+    const int pairs = p.r >> 1;
+    const int per_qt = p.B * p.G * pairs;
+    const int qt = p.n_qt - 1 - (int)(blockIdx.x / per_qt);
+    const int rem = (int)(blockIdx.x % per_qt);
+    const int b = rem / (p.G * pairs);
+    const int g = (rem / pairs) % p.G;
+    const int h0 = g * p.r + 2 * (rem % pairs);
+    const int s0 = qt * kBM;
+    const int n_kv = qt + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_ready[s], 128);
+        }
+        mbar_init(o_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 9) tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmq);
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+            const uint64_t pol_q = l2_policy_evict_first();
+            const uint64_t pol_kv = l2_policy_evict_last();
+            mbar_arrive_expect_tx(bar_q, 2 * kTile);
+            for (int hh = 0; hh < 2; ++hh)
+                for (int half = 0; half < 2; ++half)
+                    tma_load_4d(sm + kOffQ + hh * kTile + half * kHalf, &tmq, bar_q, half * 64, h0 + hh, s0,
+                                b, pol_q);
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                if (*vabort || !mbar_wait(&k_empty[st], ph ^ 1, p.timeout_ns)) {
+                    set_status(p.status, STATUS_TIMEOUT);
+                    *vabort = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(&k_full[st], kTile);
+                for (int half = 0; half < 2; ++half)
+                    tma_load_4d(sm + kOffK + st * kTile + half * kHalf, &tmk, &k_full[st], half * 64, g, j * kBN,
+                                b, pol_kv);
+                if (*vabort || !mbar_wait(&v_empty[st], ph ^ 1, p.timeout_ns)) {
+                    set_status(p.status, STATUS_TIMEOUT);
+                    *vabort = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(&v_full[st], kTile);
+                for (int half = 0; half < 2; ++half)
+                    tma_load_4d(sm + kOffV + st * kTile + half * kHalf, &tmv, &v_full[st], half * 64, g, j * kBN,
+                                b, pol_kv);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = tc::idesc_bf16(128, 128, false, false);
+            constexpr uint32_t idesc_o = tc::idesc_bf16(128, 128, false, true);
+            const uint32_t q_addr = smem_u32(sm + kOffQ), k_addr = smem_u32(sm + kOffK),
+                           v_addr = smem_u32(sm + kOffV);
+            bool issued = false, ok = true;
+            auto wait = [&](uint64_t *bar, uint32_t par) {
+                if (!ok || *vabort || !mbar_wait(bar, par, p.timeout_ns)) {
+                    if (ok) set_status(p.status, STATUS_TIMEOUT);
+                    ok = false;
+                    *vabort = 1;
+                }
+                return ok;
+            };
+            // S_h = Q_h K^T: 8 K-steps of 16 over d_h = 128 (two 64-wide swizzled halves)
+            auto issue_s = [&](int hh, int ks) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    const uint64_t a = tc::sdesc_sw128(q_addr + hh * kTile + off, 16, 1024);
+                    const uint64_t bd = tc::sdesc_sw128(k_addr + ks * kTile + off, 16, 1024);
+                    tc::mma_ss(tmem + hh * 128, a, bd, idesc_s, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_h += P_h V: 8 K-steps of 16 keys; V is MN-major (d_h contiguous)
+            auto issue_pv = [&](int hh, int vs, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t bd = tc::sdesc_sw128(v_addr + vs * kTile + kk * 2048, kHalf, 1024);
+                    tc::mma_ts(tmem + 256 + hh * 128, tmem + hh * 128 + kk * 8, bd, idesc_o,
+                               (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            if (wait(bar_q, 0) && wait(&k_full[0], 0)) {
+                issue_s(0, 0);
+                tc::commit(&s_full[0]);
+                issue_s(1, 0);
+                tc::commit(&s_full[1]);
+                tc::commit(&k_empty[0]);
+                issued = true;
+                for (int j = 0; j < n_kv && ok; ++j) {
+                    const int st = j & 1;
+                    const uint32_t ph = (j >> 1) & 1;
+                    const int st2 = (j + 1) & 1;
+                    const uint32_t ph2 = ((j + 1) >> 1) & 1;
+                    if (!wait(&v_full[st], ph) || !wait(&p_ready[0], j & 1)) break;
+                    tc::fence_after();
+                    issue_pv(0, st, j > 0);
+                    if (j + 1 < n_kv) {
+                        if (!wait(&k_full[st2], ph2)) break;
+                        issue_s(0, st2);
+                        tc::commit(&s_full[0]);
+                    }
+                    if (!wait(&p_ready[1], j & 1)) break;
+                    tc::fence_after();
+                    issue_pv(1, st, j > 0);
+                    tc::commit(&v_empty[st]);
+                    if (j + 1 < n_kv) {
+                        issue_s(1, st2);
+                        tc::commit(&s_full[1]);
+                        tc::commit(&k_empty[st2]);
+                    }
+                }
+                tc::commit(o_done);
+            }
+            if (issued && !ok) {  // let MMAs already issued finish before TMEM is freed
+                tc::commit(drain);
+                mbar_wait(drain, 0, p.timeout_ns);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ softmax + epilogue
+        const int hh = warp >> 2;                 // head of the pair
+        const int t = threadIdx.x & 127;          // query row in the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + hh * 128;
+        const uint32_t tO = tmem + lane_off + 256 + hh * 128;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const bool aborted = __any_sync(0xffffffffu, *vabort != 0);  // warp-uniform
+            if (aborted || !warp_wait(&s_full[hh], j & 1, p.timeout_ns)) {
+                if (lane == 0) set_status(p.status, STATUS_TIMEOUT);
+                *vabort = 1;
+                ok = false;
+                break;
+            }
+            tc::fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, sr[c]);
+            tc::wait_ld();
+            const bool diag = (j == n_kv - 1);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float x = __uint_as_float(sr[c][e]) * p.scale_log2;
+                    if (diag && (c * 32 + e) > t) x = -INFINITY;
+                    sr[c][e] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
+                }
+            float alpha = 1.f;
+            bool rescale = false;
+            if (j == 0) {
+                m = mx;  // key 0 is always visible, so mx is finite
+            } else {
+                const float mn = fmaxf(m, mx);
+                const bool need = mn > m + 8.f;
+                rescale = __any_sync(0xffffffffu, need);
+                if (need) {
+                    alpha = fast_exp2(m - mn);
+                    m = mn;
+                    l *= alpha;
+                }
+            }
+            // P = 2^(x - m) in bf16 pairs over the first 64 columns of this S block
+            float rs = 0.f;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = fast_exp2(__uint_as_float(sr[c4][2 * e]) - m);
+                    const float p1 = fast_exp2(__uint_as_float(sr[c4][2 * e + 1]) - m);
+                    rs += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                tc::st16(tS + c4 * 16, pk);
+            }
+            if (rescale) {  // O was last written by the P.V of tile j-1, complete by now
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t orow[16];
+                    tc::ld16(tO + c * 16, orow);
+                    tc::wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+                    tc::st16(tO + c * 16, orow);
+                }
+            }
+            l += rs;
+            tc::wait_st();
+            tc::fence_before();
+            mbar_arrive(&p_ready[hh]);
+        }
+        // epilogue: O / l -> bf16 -> out[b, s0 + t, h0 + hh, :]
+        const bool go = __all_sync(0xffffffffu, ok && *vabort == 0);
+        if (go && warp_wait(o_done, 0, p.timeout_ns)) {
+            tc::fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const int s = s0 + t;
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) +
+                                 (((size_t)b * p.S + s) * p.H + h0 + hh) * 128;
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+                uint32_t orow[16];
+                tc::ld16(tO + c * 16, orow);
+                tc::wait_ld();
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    pk[e] = pack_bf16x2(__uint_as_float(orow[2 * e]) * inv, __uint_as_float(orow[2 * e + 1]) * inv);
+                if (s < p.S) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 16);
+                    d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+        } else if (lane == 0) {
+            set_status(p.status, STATUS_TIMEOUT);
+        }
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc::fence_after();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const CUtensorMap *tmk,
+                           const CUtensorMap *tmv, cudaStream_t st) {
+    PrefillParams p = {};
+    p.out = a.out;
+    p.status = a.status;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.B = a.B;
+    p.S = a.S;
+    p.H = a.H;
+    p.G = a.G;
+    p.r = a.H / a.G;
+    p.n_qt = (a.S + kBM - 1) / kBM;
+    p.timeout_ns = a.timeout_ns;
+    const long long grid = (long long)p.n_qt * a.B * a.G * (p.r / 2);
+    if (grid <= 0 || grid >= (1ll << 31)) return cudaErrorInvalidConfiguration;
+    cudaError_t e = cudaFuncSetAttribute(prefill_causal_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    prefill_causal_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(*tmq, *tmk, *tmv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace gqa

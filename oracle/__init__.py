@@ -110,10 +110,12 @@ def _i32(x):
     return t, t.data_ptr()
 
 
-def _rows(rows):
+def _rows(rows, limit):
     if rows is None:
         return None, None, 0
     t = torch.as_tensor(rows, dtype=torch.int64).reshape(-1).contiguous()
+    if t.numel() and (int(t.min()) < 0 or int(t.max()) >= limit):
+        raise IndexError("row index outside [0, %d)" % limit)
     return t, t.data_ptr(), t.numel()
 
 
@@ -144,7 +146,7 @@ def gqa_decode(q, k_cache, v_cache, seqlens, scale, rows=None, nthreads=0):
     B, H, d_h = qt.shape
     _, G, T_cap, _ = kt.shape
     st, sp = _i32(seqlens)
-    rt, rp, nr = _rows(rows)
+    rt, rp, nr = _rows(rows, B * H)
     out = torch.empty((nr, d_h) if rt is not None else (B, H, d_h), dtype=torch.float64)
     rc = lib.oracle_gqa_decode(qp, qdt, kp, vp_, kdt, sp, float(scale), out.data_ptr(),
                                B, H, G, d_h, T_cap, rp, nr, int(nthreads))
@@ -186,7 +188,7 @@ def gqa_prefill_causal(q, k, v, scale, rows=None, nthreads=0):
         raise TypeError("q, k, v must share a dtype")
     B, S, H, d_h = qt.shape
     G = kt.shape[2]
-    rt, rp, nr = _rows(rows)
+    rt, rp, nr = _rows(rows, B * S * H)
     out = torch.empty((nr, d_h) if rt is not None else (B, S, H, d_h), dtype=torch.float64)
     rc = lib.oracle_gqa_prefill_causal(qp, kp, vp_, qdt, float(scale), out.data_ptr(),
                                        B, S, H, G, d_h, rp, nr, int(nthreads))

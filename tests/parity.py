@@ -1,0 +1,48 @@
+"""Tolerances for comparing kernel outputs (as stored) with the fp64 oracle.
+
+bf16 inputs with fp32 accumulation: max abs error 2e-3 and max relative error
+1e-2; fp32 inputs: 1e-5 for both.  Two readings are used:
+
+* ``assert_strict``: max_i |d_i| <= atol AND max_i |d_i| / max_i |ref_i| <= rtol
+  (normwise relative).  Used at the benchmark workloads, whose outputs are
+  small averages (|out| << 1).
+* ``assert_close``: |d_i| <= atol + rtol * |ref_i| for every i.  Used in the
+  sweeps, where a short sequence makes |out| ~ 1 and rounding the output to
+  bf16 alone moves it by up to 2^-9 |out| > 2e-3.
+Every value must be finite.
+"""
+import torch
+
+TOL = {torch.bfloat16: (2e-3, 1e-2), torch.float32: (1e-5, 1e-5)}
+
+
+def errors(got, ref):
+    got = got.detach().double().cpu()
+    ref = ref.detach().double().cpu()
+    d = (got - ref).abs()
+    if d.numel() == 0:
+        return 0.0, 0.0
+    maxabs = d.max().item()
+    refmax = ref.abs().max().item()
+    return maxabs, (maxabs / refmax if refmax > 0 else maxabs)
+
+
+def assert_strict(got, ref, dtype):
+    atol, rtol = TOL[dtype]
+    g = got.detach().double().cpu()
+    assert torch.isfinite(g).all(), "non-finite output"
+    maxabs, normrel = errors(got, ref)
+    assert maxabs <= atol and normrel <= rtol, (maxabs, normrel)
+    return maxabs, normrel
+
+
+def assert_close(got, ref, dtype):
+    atol, rtol = TOL[dtype]
+    g = got.detach().double().cpu()
+    r = ref.detach().double().cpu()
+    assert torch.isfinite(g).all(), "non-finite output"
+    d = (g - r).abs()
+    bad = d > atol + rtol * r.abs()
+    assert not bad.any(), "max excess %g at %s" % ((d - atol - rtol * r.abs()).max().item(),
+                                                   bad.nonzero()[:4].tolist())
+    return errors(got, ref)

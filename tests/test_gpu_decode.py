@@ -1,0 +1,148 @@
+"""GQA decode through the C ABI vs the fp64 oracle on the same seeded inputs.
+
+Sweeps cover d_h in {64, 128}, group sizes H/G from 1 (MHA) to 64, ragged
+lengths (0, 1, tile boundaries 63/64/65, non-multiples), NaN-poisoned cache
+padding, split counts from 1 to more CTAs than tiles, fp32 and bf16.  The
+benchmark workloads run at full size: every row for the 7B-shaped step,
+sampled rows for the 70B-shaped ragged step and the 131072-token G sweep.
+"""
+import math
+
+import pytest
+import torch
+
+import gqa_inputs as gi
+import oracle
+from parity import assert_close, assert_strict
+
+pytestmark = pytest.mark.gpu
+
+
+def run_decode(gqa, x, stream=None):
+    q, k, v = x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda()
+    sl = x.seqlens.to(torch.int32).cuda()
+    out = gqa.decode(q, k, v, sl, x.scale, stream=stream)
+    gqa.get_status()
+    return out.cpu()
+
+
+def test_tiny_fp32_workload(gqa):
+    x = gi.workload_inputs("tiny_decode_fp32")
+    assert x.scale == 1.0 / 8.0
+    got = run_decode(gqa, x)
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    assert_strict(got, ref, torch.float32)
+
+
+@pytest.mark.parametrize("d_h", [64, 128])
+@pytest.mark.parametrize("r", [1, 2, 4, 8, 12, 16, 24, 32, 64])
+def test_bf16_group_sizes(gqa, d_h, r):
+    G = 2
+    x = gi.decode_inputs(6, r * G, G, d_h, 200, torch.bfloat16, seed=100 + r,
+                         seqlens=[200, 1, 64, 65, 0, 137])
+    got = run_decode(gqa, x)
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    assert_close(got, ref, torch.bfloat16)
+    assert torch.equal(got[4], torch.zeros_like(got[4]))  # empty cache row
+
+
+@pytest.mark.parametrize("d_h", [64, 128])
+@pytest.mark.parametrize("r", [1, 3, 8])
+def test_f32_sweep(gqa, d_h, r):
+    G = 3
+    x = gi.decode_inputs(4, r * G, G, d_h, 97, torch.float32, seed=200 + r,
+                         seqlens=[97, 1, 33, 64])
+    got = run_decode(gqa, x)
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    assert_close(got, ref, torch.float32)
+
+
+@pytest.mark.parametrize("ctas", [1, 2, 3, 7, 50, 1000])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_forced_split_counts(gqa, monkeypatch, ctas, dtype):
+    """Shares that start mid-segment and span several segments."""
+    monkeypatch.setenv("GQA_DECODE_CTAS", str(ctas))
+    x = gi.decode_inputs(5, 16, 4, 128, 300, dtype, seed=300, seqlens=[300, 1, 0, 129, 64])
+    got = run_decode(gqa, x)
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    assert_close(got, ref, dtype)
+
+
+def test_seqlens_out_of_range_are_clamped_and_flagged(gqa):
+    x = gi.decode_inputs(3, 8, 2, 64, 100, torch.bfloat16, seed=400, seqlens=[100, 50, 10],
+                         nan_pad=False)
+    q, k, v = x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda()
+    sl = torch.tensor([130, -5, 10], dtype=torch.int32, device="cuda")
+    out = gqa.decode(q, k, v, sl, x.scale)
+    with pytest.raises(gqa.GQAError) as ei:
+        gqa.get_status()
+    assert ei.value.code == -7
+    gqa.get_status()  # cleared
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, [100, 0, 10], x.scale)
+    assert_close(out.cpu(), ref, torch.bfloat16)
+
+
+def test_deterministic_and_stream_ordered(gqa):
+    x = gi.decode_inputs(4, 32, 8, 128, 1000, torch.bfloat16, seed=500, ragged=(1, 1000))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a = run_decode(gqa, x, stream=s)
+        b = run_decode(gqa, x, stream=s)
+    assert torch.equal(a, b)
+
+
+def test_gqa_equals_mha_on_repeated_kv(gqa):
+    """The page's broadcast identity, on the GPU: G heads shared by H/G query
+    heads gives the MHA result on K/V repeated H/G times."""
+    x = gi.decode_inputs(2, 16, 4, 128, 256, torch.bfloat16, seed=600, seqlens=[256, 77])
+    got = run_decode(gqa, x)
+    xr = gi.DecodeInputs(x.q, x.k_cache.repeat_interleave(4, dim=1).contiguous(),
+                         x.v_cache.repeat_interleave(4, dim=1).contiguous(), x.seqlens,
+                         x.scale, 2, 16, 16, 128, 256)
+    mha = run_decode(gqa, xr)
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    assert_close(got, ref, torch.bfloat16)
+    assert_close(mha, ref, torch.bfloat16)
+
+
+# ------------------------------------------------------------ full-size workloads
+
+def test_llama2_7b_decode_full(gqa):
+    """B=16, H=32, G=8, d_h=128, T=4096, bf16: every output row."""
+    x = gi.workload_inputs("llama2_7b_decode")
+    got = run_decode(gqa, x)
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    assert_strict(got, ref, torch.bfloat16)
+
+
+def test_llama2_70b_ragged_decode_full(gqa):
+    """B=32, H=64, G=8, d_h=128, T_b uniform in [1024, 8192], NaN padding."""
+    x = gi.workload_inputs("llama2_70b_ragged_decode")
+    assert int(x.seqlens.min()) >= 1024 and int(x.seqlens.max()) <= 8192
+    got = run_decode(gqa, x)
+    assert torch.isfinite(got.float()).all()
+    gen = torch.Generator().manual_seed(1)
+    rows = sorted(set(torch.randint(0, 32 * 64, (192,), generator=gen).tolist()
+                      + [0, 63, 64, 32 * 64 - 1]))
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, rows=rows)
+    assert_strict(got.reshape(-1, 128)[rows], ref, torch.bfloat16)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32])
+def test_long_context_decode_full(gqa, G):
+    """B=4, H=32, d_h=128, T=131072: sampled rows of sequences 0 and 3."""
+    x = gi.decode_inputs(4, 32, G, 128, 131072, torch.bfloat16, seed=0, device="cuda")
+    out = gqa.decode(x.q, x.k_cache, x.v_cache, x.seqlens.cuda(), x.scale)
+    gqa.get_status()
+    out = out.cpu()
+    assert torch.isfinite(out.float()).all()
+    r = 32 // G
+    for b in (0, 3):
+        heads = sorted({h for h in (0, r - 1, r, 31, (7 * b + 5) % 32, (11 * b + 17) % 32)
+                        if h < 32})
+        kb = x.k_cache[b:b + 1].cpu()
+        vb = x.v_cache[b:b + 1].cpu()
+        ref = oracle.gqa_decode(x.q[b:b + 1].cpu(), kb, vb, x.seqlens[b:b + 1], x.scale,
+                                rows=heads)
+        assert_strict(out[b, heads], ref, torch.bfloat16)
+        del kb, vb

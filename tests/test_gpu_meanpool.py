@@ -1,0 +1,62 @@
+"""Mean-pool init through the C ABI vs the oracle: bit-exact (same binary64
+operations in the same order, one nearest-even rounding)."""
+import pytest
+import torch
+
+import gqa_inputs as gi
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def bits(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+
+
+def run(gqa, wk, wv, G):
+    ok, ov = gqa.meanpool_kv(wk.cuda(), wv.cuda(), G)
+    gqa.get_status()
+    return ok.cpu(), ov.cpu()
+
+
+def test_meanpool_full_workload_bit_exact(gqa):
+    """W_K, W_V [64, 128, 8192] bf16 ~ N(0, 0.02) into 8 groups."""
+    wk, wv = gi.workload_inputs("meanpool_init")
+    ok, ov = run(gqa, wk, wv, 8)
+    assert torch.equal(bits(ok), bits(oracle.meanpool(wk, 8)))
+    assert torch.equal(bits(ov), bits(oracle.meanpool(wv, 8)))
+
+
+@pytest.mark.parametrize("H,G,d_h,d", [(8, 2, 4, 16), (12, 4, 3, 5), (16, 16, 8, 8),
+                                       (32, 1, 8, 24), (6, 2, 7, 9), (64, 8, 128, 64)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_meanpool_shapes_bit_exact(gqa, H, G, d_h, d, dtype):
+    wk, wv = gi.meanpool_inputs(H, d_h, d, dtype=dtype, seed=H * 31 + d, std=0.5)
+    ok, ov = run(gqa, wk, wv, G)
+    assert torch.equal(bits(ok), bits(oracle.meanpool(wk, G)))
+    assert torch.equal(bits(ov), bits(oracle.meanpool(wv, G)))
+
+
+def test_meanpool_integer_coded(gqa):
+    H, G = 16, 4
+    e = torch.arange(8 * 16, dtype=torch.float32).reshape(8, 16) % 16
+    W = (16.0 * torch.arange(H, dtype=torch.float32)[:, None, None] + e[None]).to(torch.bfloat16)
+    ok, ov = run(gqa, W, W.flip(0).contiguous(), G)
+    r = H // G
+    for g in range(G):
+        exp = sum(W[g * r + j].double() for j in range(r)) / r
+        assert torch.equal(ok[g].double(), oracle.round_to(exp, torch.bfloat16).double())
+
+
+def test_meanpool_unaligned_views(gqa):
+    """Element offsets that break 16-byte alignment take the element-wise kernel."""
+    H, G, d_h, d = 8, 2, 5, 7
+    base = torch.randn(2 * H * d_h * d + 3, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    dev = base.cuda()
+    n = H * d_h * d
+    wk = dev[1:1 + n].view(H, d_h, d)
+    wv = dev[2 + n:2 + 2 * n].view(H, d_h, d)
+    ok, ov = gqa.meanpool_kv(wk, wv, G)
+    gqa.get_status()
+    assert torch.equal(bits(ok.cpu()), bits(oracle.meanpool(wk.cpu(), G)))
+    assert torch.equal(bits(ov.cpu()), bits(oracle.meanpool(wv.cpu(), G)))

@@ -1,0 +1,71 @@
+"""Causal GQA prefill (tcgen05) through the C ABI vs the fp64 oracle.
+
+Ordered from one CTA (one 128-row query tile, diagonal KV tile only) up to the
+full B=2, S=8192, H=64, G=8 workload (sampled rows).  Ragged S (not a multiple
+of the 128-row tile) and several group sizes are covered.
+"""
+import pytest
+import torch
+
+import gqa_inputs as gi
+import oracle
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run(gqa, x):
+    out = gqa.prefill_causal(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.scale)
+    gqa.get_status()
+    return out.cpu()
+
+
+@pytest.mark.parametrize("B,S,H,G", [
+    (1, 128, 2, 1),      # one CTA, diagonal tile only
+    (1, 256, 2, 1),      # two query tiles, one and two KV tiles
+    (1, 384, 4, 2),
+    (2, 200, 8, 2),      # ragged: 200 = 128 + 72
+    (1, 1, 2, 1),        # a single position
+    (1, 129, 4, 1),      # one row past a tile
+    (2, 77, 16, 2),      # r = 8
+    (1, 1000, 8, 4),     # r = 2
+    (1, 640, 32, 1),     # r = 32 (MQA-like)
+])
+def test_prefill_small(gqa, B, S, H, G):
+    x = gi.prefill_inputs(B, S, H, G, 128, torch.bfloat16, seed=S + 7 * H)
+    got = run(gqa, x)
+    ref = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale)
+    assert_close(got, ref, torch.bfloat16)
+
+
+def test_prefill_deterministic(gqa):
+    x = gi.prefill_inputs(1, 512, 8, 2, 128, torch.bfloat16, seed=3)
+    assert torch.equal(run(gqa, x), run(gqa, x))
+
+
+def test_prefill_last_row_matches_decode(gqa):
+    """Last prefill row over S keys equals one decode step over the same K/V."""
+    x = gi.prefill_inputs(2, 300, 8, 2, 128, torch.bfloat16, seed=5)
+    pre = run(gqa, x)
+    kc = x.k.permute(0, 2, 1, 3).contiguous()
+    vc = x.v.permute(0, 2, 1, 3).contiguous()
+    dec = gqa.decode(x.q[:, -1].contiguous().cuda(), kc.cuda(), vc.cuda(),
+                     torch.tensor([300, 300], dtype=torch.int32, device="cuda"), x.scale).cpu()
+    ref = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale)[:, -1]
+    assert_close(pre[:, -1], ref, torch.bfloat16)
+    assert_close(dec, ref, torch.bfloat16)
+
+
+def test_causal_prefill_full_workload(gqa):
+    """B=2, S=8192, H=64, G=8, d_h=128: rows at tile edges and random rows."""
+    x = gi.workload_inputs("causal_prefill")
+    got = run(gqa, x)
+    assert torch.isfinite(got.float()).all()
+    S, H = 8192, 64
+    gen = torch.Generator().manual_seed(11)
+    picks = [(0, 0, 0), (1, 8191, 63), (0, 127, 5), (0, 128, 9), (1, 4095, 33), (1, 4096, 40)]
+    for s in torch.randint(0, S, (160,), generator=gen).tolist():
+        picks.append((s % 2, s, int(torch.randint(0, H, (1,), generator=gen))))
+    rows = [(b * S + s) * H + i for b, s, i in picks]
+    ref = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, rows=rows)
+    assert_close(got.reshape(-1, 128)[rows], ref, torch.bfloat16)

@@ -372,3 +372,12 @@ def test_round_f32():
     got = oracle.round_to(xs, torch.float32)
     assert got[0].item() == 1.0 and got[1].item() == 1.0 + 2 ** -22
     assert got[2].item() == 2 ** -149 and math.isinf(got[3].item())
+
+
+def test_row_selection_rejects_out_of_range():
+    x = gi.decode_inputs(1, 4, 2, 8, 8, torch.float32, seed=18)
+    with pytest.raises(IndexError):
+        oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, rows=[4])
+    p = gi.prefill_inputs(1, 4, 2, 1, 8, torch.float32, seed=18)
+    with pytest.raises(IndexError):
+        oracle.gqa_prefill_causal(p.q, p.k, p.v, p.scale, rows=[-1])
