@@ -41,6 +41,7 @@ constexpr int kCWarps = 4;      // consumer warps
 constexpr int kThreads = (kCWarps + 1) * 32;
 constexpr int kHalfBytes = kTile * 128;  // one [64 tokens x 64 dims] bf16 box
 constexpr int kThreadsF32 = 128;
+constexpr int kSplitPMaxLen = 256;  // sequences this short carry P as two bf16 terms
 
 struct DecodeParams {
     const void *q;
@@ -235,7 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
         const int b = c.b, bg = c.b * p.G + c.g;
         const int t0 = c.j * kTile;
-        const int n_valid = min(kTile, clamp_len(p.seqlens[b], p.T_cap) - t0);
+        const int seq_len = clamp_len(p.seqlens[b], p.T_cap);
+        const int n_valid = min(kTile, seq_len - t0);
         if (bg != cur_bg) {  // first tile of a piece: this group's queries
             cur_bg = bg;
             const int hl_a = mt * 16 + g8, hl_b = hl_a + 8;
@@ -335,7 +337,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     o[nn][2] *= al_b;
                     o[nn][3] *= al_b;
                 }
-                // O[16 x D] += P[16 x 16] . V[16 x D]
+                // O[16 x D] += P[16 x 16] . V[16 x D].  For short sequences the bf16
+                // rounding of P does not average out; there P is carried as two bf16
+                // terms P_hi + P_lo (about 16 significant bits).
+                const bool split_p = seq_len <= kSplitPMaxLen;
+                uint32_t pl[4] = {0u, 0u, 0u, 0u};
+                if (split_p) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const float2 ha = unpack_bf16x2(pa[2 * nt + 0]);
+                        const float2 hb = unpack_bf16x2(pa[2 * nt + 1]);
+                        pl[2 * nt + 0] = pack_bf16x2(fast_exp2(sc[nt][0] - mu_a) - ha.x,
+                                                     fast_exp2(sc[nt][1] - mu_a) - ha.y);
+                        pl[2 * nt + 1] = pack_bf16x2(fast_exp2(sc[nt][2] - mu_b) - hb.x,
+                                                     fast_exp2(sc[nt][3] - mu_b) - hb.y);
+                    }
+                }
                 {
                     const int tok = row0 + (((lane >> 3) & 1) << 3) + (lane & 7);
                     const int dsel = (lane >> 4) << 3;
@@ -345,6 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ldsm_x4_t(vbase + swz(tok, n2 * 16 + dsel), b0, b1, b2, b3);
                         mma_16816(o[2 * n2], pa, b0, b1);
                         mma_16816(o[2 * n2 + 1], pa, b2, b3);
+                        if (split_p) {
+                            mma_16816(o[2 * n2], pl, b0, b1);
+                            mma_16816(o[2 * n2 + 1], pl, b2, b3);
+                        }
                     }
                 }
             }

@@ -17,6 +17,7 @@
 //   warps 0-3   softmax + epilogue for head 0 (one thread per query row =
 //   warps 4-7   one TMEM lane), head 1.  While one group runs its softmax the
 //               tensor core works on the other head's MMAs.
+//   warps 10-11 idle (they complete the third warpgroup for the register split).
 // TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,384) O0, [384,512) O1.
 // P (bf16) overwrites the first 64 columns of its S block after S is read.
 // Online softmax in the base-2 domain; the running max is only moved (and O
@@ -37,7 +38,16 @@ constexpr int kBM = 128;                 // query rows per tile
 constexpr int kBN = 128;                 // keys per KV tile
 constexpr int kHalf = 128 * 64 * 2;      // one [128 rows x 64 bf16] swizzled box
 constexpr int kTile = 2 * kHalf;         // [128 x 128] bf16
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;           // 3 warpgroups
+// Register split (setmaxnreg): the launch gives every thread kLaunchRegs; the
+// TMA/MMA warpgroup then drops to kLowRegs and the two softmax warpgroups rise
+// to kHighRegs.  2*128*kHighRegs + 128*kLowRegs must not exceed
+// 384*kLaunchRegs, or an .inc would wait for registers that never come; the
+// launcher checks the compiled register count against this before launching.
+constexpr int kLaunchRegs = 168;
+constexpr int kLowRegs = 88;
+constexpr int kHighRegs = 208;
+static_assert(2 * 128 * kHighRegs + 128 * kLowRegs <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kOffQ = 0;                 // Q0, Q1
 constexpr int kOffK = 2 * kTile;         // K stages 0, 1
@@ -123,7 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
+    if (warp >= 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+      if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tmq);
@@ -160,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 9) {
+      } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = tc::idesc_bf16(128, 128, false, false);
@@ -176,24 +188,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return ok;
             };
+            // Descriptors are built from one base per operand; a K-step only moves the
+            // start address (low word, 16-byte units).  The loops stay rolled so the
+            // issuing warp needs few registers.
+            const uint64_t dq = tc::sdesc_sw128(q_addr, 16, 1024);
+            const uint64_t dk = tc::sdesc_sw128(k_addr, 16, 1024);
+            const uint64_t dv = tc::sdesc_sw128(v_addr, kHalf, 1024);
             // S_h = Q_h K^T: 8 K-steps of 16 over d_h = 128 (two 64-wide swizzled halves)
             auto issue_s = [&](int hh, int ks) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    const uint64_t a = tc::sdesc_sw128(q_addr + hh * kTile + off, 16, 1024);
-                    const uint64_t bd = tc::sdesc_sw128(k_addr + ks * kTile + off, 16, 1024);
-                    tc::mma_ss(tmem + hh * 128, a, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+                    tc::mma_ss(tmem + hh * 128, dq + ((hh * kTile) >> 4) + off, dk + ((ks * kTile) >> 4) + off,
+                               idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_h += P_h V: 8 K-steps of 16 keys; V is MN-major (d_h contiguous)
+            // O_h += P_h V: 8 K-steps of 16 keys; V is MN-major (d_h contiguous).  On
+            // the first query tile a second pass adds P_lo (TMEM columns 64..127).
             auto issue_pv = [&](int hh, int vs, bool acc) {
+                const int passes = qt == 0 ? 2 : 1;
+#pragma unroll 1
+                for (int ps = 0; ps < passes; ++ps)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t bd = tc::sdesc_sw128(v_addr + vs * kTile + kk * 2048, kHalf, 1024);
-                    tc::mma_ts(tmem + 256 + hh * 128, tmem + hh * 128 + kk * 8, bd, idesc_o,
-                               (acc || kk > 0) ? 1u : 0u);
-                }
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_ts(tmem + 256 + hh * 128, tmem + hh * 128 + ps * 64 + kk * 8,
+                                   dv + ((vs * kTile + kk * 2048) >> 4), idesc_o,
+                                   (acc || ps > 0 || kk > 0) ? 1u : 0u);
             };
             if (wait(bar_q, 0) && wait(&k_full[0], 0)) {
                 issue_s(0, 0);
@@ -233,7 +253,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
+      }
+      // warps 10 and 11: spare members of the TMA/MMA warpgroup
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
         // ------------------------------------------------ softmax + epilogue
         const int hh = warp >> 2;                 // head of the pair
         const int t = threadIdx.x & 127;          // query row in the tile = TMEM lane
@@ -242,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tO = tmem + lane_off + 256 + hh * 128;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
+        const bool split_p = (qt == 0);
         for (int j = 0; j < n_kv; ++j) {
             const bool aborted = __any_sync(0xffffffffu, *vabort != 0);  // warp-uniform
             if (aborted || !warp_wait(&s_full[hh], j & 1, p.timeout_ns)) {
@@ -280,19 +304,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l *= alpha;
                 }
             }
-            // P = 2^(x - m) in bf16 pairs over the first 64 columns of this S block
+            // P = 2^(x - m) in bf16 pairs over the first 64 columns of this S block.
+            // Rows of the first query tile see at most 128 keys, too few for the bf16
+            // rounding of P to average out; there P is carried as P_hi + P_lo (two bf16
+            // terms, about 16 significant bits), P_lo in columns 64..127.
             float rs = 0.f;
+            if (!split_p) {
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t pk[16];
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(__uint_as_float(sr[c4][2 * e]) - m);
-                    const float p1 = fast_exp2(__uint_as_float(sr[c4][2 * e + 1]) - m);
-                    rs += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = fast_exp2(__uint_as_float(sr[c4][2 * e]) - m);
+                        const float p1 = fast_exp2(__uint_as_float(sr[c4][2 * e + 1]) - m);
+                        rs += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tc::st16(tS + c4 * 16, pk);
                 }
-                tc::st16(tS + c4 * 16, pk);
+            } else {  // first query tile: P_hi to columns 0..63, P_lo to 64..127
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        uint32_t ph[4], pl[4];
+#pragma unroll
+                        for (int e1 = 0; e1 < 4; ++e1) {
+                            const int e = e4 * 4 + e1;
+                            const float p0 = fast_exp2(__uint_as_float(sr[c4][2 * e]) - m);
+                            const float p1 = fast_exp2(__uint_as_float(sr[c4][2 * e + 1]) - m);
+                            rs += p0 + p1;
+                            ph[e1] = pack_bf16x2(p0, p1);
+                            const float2 h = unpack_bf16x2(ph[e1]);
+                            pl[e1] = pack_bf16x2(p0 - h.x, p1 - h.y);
+                        }
+                        tc::st4(tS + c4 * 16 + e4 * 4, ph);
+                        tc::st4(tS + 64 + c4 * 16 + e4 * 4, pl);
+                    }
+                }
             }
             if (rescale) {  // O was last written by the P.V of tile j-1, complete by now
 #pragma unroll 1
@@ -362,8 +411,11 @@ cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const C
     p.timeout_ns = a.timeout_ns;
     const long long grid = (long long)p.n_qt * a.B * a.G * (p.r / 2);
     if (grid <= 0 || grid >= (1ll << 31)) return cudaErrorInvalidConfiguration;
-    cudaError_t e = cudaFuncSetAttribute(prefill_causal_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_causal_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split would not hold
+    e = cudaFuncSetAttribute(prefill_causal_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     prefill_causal_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(*tmq, *tmk, *tmv, p);
     return cudaGetLastError();
