@@ -110,6 +110,35 @@ GQA_API int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                size_t workspace_bytes, gqa_stream_t stream);
 
 /*
+ * gqa_decode_noalloc -- gqa_decode for callers that cannot allocate device
+ * memory.  (The pages have no counterpart: this is a deployment convenience.)
+ *
+ * gqa_decode needs scratch for its per-split partial results, which its caller
+ * allocates.  Some callers cannot: a plug-in inside a host runtime that has
+ * already reserved the device's memory for its own allocator, or a serving loop
+ * that must not allocate after start-up because an allocation could stall or
+ * fail it.  This entry point takes the same arguments as gqa_decode minus the
+ * workspace and uses a scratch array compiled into the library instead:
+ *   - the array holds GQA_DECODE_NOALLOC_SCRATCH_BYTES (8 MiB) and stays
+ *     resident on every GPU that loads the library until the process exits;
+ *   - shapes whose scratch (gqa_decode_workspace_bytes) exceeds it are rejected
+ *     with GQA_ERR_WORKSPACE before anything is launched;
+ *   - the first call on a device looks up the array's device address on that
+ *     device (a one-time set-up); make that first call before any stream
+ *     capture;
+ *   - all calls on a device share the one array: two calls whose kernels can
+ *     overlap on the GPU (different streams with no ordering) race on it;
+ *   - the array keeps the last call's contents; nothing in it needs to start
+ *     at zero, since each call writes every record it reads.
+ * It never calls cudaMalloc, cudaFree or any allocating routine.  Results are
+ * those of gqa_decode on the same inputs.
+ */
+#define GQA_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+GQA_API int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *seqlens, float scale, void *out, int B, int H,
+                               int G, int d_h, int T_cap, gqa_dtype dt, gqa_stream_t stream);
+
+/*
  * gqa_prefill_causal -- causal GQA attention over a whole prompt: for each b,
  * position s and query head i,
  *     out[b,s,i,:] = sum_{t <= s} softmax_t(scale * <q[b,s,i,:], k[b,t,g,:]>) v[b,t,g,:]

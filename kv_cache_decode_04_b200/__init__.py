@@ -22,7 +22,7 @@ import os
 
 import torch
 
-__all__ = ["decode", "decode_workspace_bytes", "prefill_causal", "meanpool_kv",
+__all__ = ["decode", "decode_noalloc", "decode_workspace_bytes", "prefill_causal", "meanpool_kv",
            "kv_cache_bytes", "get_status", "GQAError", "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqa.so")
@@ -33,7 +33,7 @@ _ERRORS = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGN", -4: "CUDA", -5: "WORKS
 
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_kv_cache_bytes", "gqa_decode_workspace_bytes", "gqa_decode",
-           "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_status",
+           "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_status",
            "gqa_last_error_string", "gqa_version")
 
 
@@ -55,6 +55,8 @@ def _load():
     L.gqa_decode_workspace_bytes.restype = sz
     L.gqa_decode.argtypes = [vp, vp, vp, vp, f32, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]
     L.gqa_decode.restype = i32
+    L.gqa_decode_noalloc.argtypes = [vp, vp, vp, vp, f32, vp, i32, i32, i32, i32, i32, i32, vp]
+    L.gqa_decode_noalloc.restype = i32
     L.gqa_prefill_causal.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, vp]
     L.gqa_prefill_causal.restype = i32
     L.gqa_meanpool_kv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
@@ -135,6 +137,32 @@ def decode(q, k_cache, v_cache, seqlens, scale=None, out=None, workspace=None, s
                         _dev(seqlens, "seqlens"), float(scale), _dev(out, "out"), B, H, G, d_h,
                         T_cap, code, _dev(workspace, "workspace"), workspace.numel(),
                         _stream(stream))
+    _check(rc)
+    return out
+
+
+def decode_noalloc(q, k_cache, v_cache, seqlens, scale=None, out=None, stream=None):
+    """Same as :func:`decode`, with the library's built-in scratch instead of a workspace.
+
+    For callers that cannot allocate device memory; see gqa_decode_noalloc in
+    include/gqa.h for the size limit and the sharing rules of that scratch.
+    """
+    B, H, d_h = q.shape
+    Bk, G, T_cap, dk = k_cache.shape
+    if Bk != B or dk != d_h or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between q, k_cache and v_cache")
+    if q.dtype != k_cache.dtype or q.dtype != v_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share a dtype")
+    if seqlens.dtype != torch.int32 or seqlens.numel() != B:
+        raise ValueError("seqlens must be int32 [B]")
+    code = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_h)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib.gqa_decode_noalloc(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                _dev(seqlens, "seqlens"), float(scale), _dev(out, "out"), B, H, G,
+                                d_h, T_cap, code, _stream(stream))
     _check(rc)
     return out
 

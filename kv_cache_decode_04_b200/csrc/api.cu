@@ -133,6 +133,8 @@ int check_dims(int B, int H, int G, int d_h) {
 
 }  // namespace
 
+int gqa::set_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
 extern "C" {
 
 int gqa_version(void) { return 100; }

@@ -54,6 +54,9 @@ struct PrefillArgs {
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const CUtensorMap *tmk,
                            const CUtensorMap *tmv, cudaStream_t stream);
 
+// Records `msg` as the calling thread's last error and returns `code`.
+int set_error(int code, const char *msg);
+
 // Mean-pool init.
 cudaError_t launch_meanpool(const void *wk, const void *wv, void *ok, void *ov, int H, int G,
                             long long n, int dtype, int num_sms, cudaStream_t stream);
