@@ -39,9 +39,14 @@ HEADLINE = "llama2_7b_decode"
 ROW_WORKLOADS = ["tiny_decode_fp32", "llama2_70b_ragged_decode"] + \
     ["long_ctx_decode_G%d" % g for g in (1, 2, 4, 8, 16, 32)] + ["causal_prefill", "meanpool_init"]
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu captures of
-# the current kernels (None until captured for the current kernel build).
-NCU_TRAFFIC = {}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch, bytes, from ncu
+# captures of the current kernels (profiles/*.md); a workload missing here has
+# no capture of its current kernel.
+NCU_TRAFFIC = {
+    "llama2_7b_decode": 273662976,      # profiles/decode_split_llama2_7b.md (split kernel)
+    "causal_prefill": 395047936,        # profiles/prefill_causal.md, half-length case x 4
+    "meanpool_init": 288346112,         # profiles/meanpool_init.md
+}
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 

@@ -29,6 +29,9 @@ WORKLOADS = {
                            dtype=torch.bfloat16),
     "meanpool_init": dict(kind="meanpool", H=64, G=8, d_h=128, d=8192,
                           dtype=torch.bfloat16, std=0.02),
+    # half-length prefill (150 MB of q/k/v/out, above the 126 MB L2) for profiler captures
+    "causal_prefill_profile": dict(kind="prefill", B=1, S=4096, H=64, G=8, d_h=128,
+                                   dtype=torch.bfloat16),
 }
 
 _CHUNK = 1 << 24  # draw at most this many normals at a time
