@@ -130,8 +130,8 @@ def decode(q, k_cache, v_cache, seqlens, scale=None, out=None, workspace=None, s
         scale = 1.0 / math.sqrt(d_h)
     if out is None:
         out = torch.empty_like(q)
-    need = decode_workspace_bytes(B, H, G, d_h, T_cap, q.dtype)
-    if workspace is None:
+    if workspace is None:  # (a given workspace's size is checked by the library)
+        need = decode_workspace_bytes(B, H, G, d_h, T_cap, q.dtype)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     rc = lib.gqa_decode(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
                         _dev(seqlens, "seqlens"), float(scale), _dev(out, "out"), B, H, G, d_h,

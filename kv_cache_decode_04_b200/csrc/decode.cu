@@ -26,6 +26,8 @@
 // warp-level bf16 tensor-core MMAs (scores, then P.V with P rounded to bf16)
 // and an fp32 online softmax; query rows are padded to 16 per MMA tile.
 // fp32 path: CUDA-core fp32 arithmetic throughout (no TF32).
+#include <atomic>
+
 #include "common.cuh"
 #include "gqa.h"
 #include "internal.h"
@@ -36,7 +38,8 @@ namespace {
 
 constexpr int kTile = 64;       // tokens per K/V tile, bf16 path
 constexpr int kTileF32 = 32;    // tokens per tile, fp32 path
-constexpr int kStages = 4;      // TMA ring depth
+constexpr int kStages = 2;      // TMA ring depth per CTA
+constexpr int kCtasPerSm = 2;   // resident split CTAs per SM (2 x 2 stages in flight)
 constexpr int kCWarps = 4;      // consumer warps
 constexpr int kThreads = (kCWarps + 1) * 32;
 constexpr int kHalfBytes = kTile * 128;  // one [64 tokens x 64 dims] bf16 box
@@ -62,10 +65,11 @@ __device__ __forceinline__ int clamp_len(int T, int T_cap) {
 }
 
 // cu[b] = G * sum_{b' < b} ceil(T_b' / TILE), T clamped to [0, T_cap];
-// cu[B] = total tiles W.  Every thread of the block must call it.
+// cu[B] = total tiles W.  Every thread of the block must call it; blockDim.x
+// is a multiple of 32 and scratch holds 32 ints.
 template <int TILE>
 __device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, bool report) {
-    const int nt = blockDim.x, tid = threadIdx.x;
+    const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int chunk = (p.B + nt - 1) / nt;
     const int b0 = min(p.B, tid * chunk), b1 = min(p.B, b0 + chunk);
     int local = 0;
@@ -76,19 +80,28 @@ __device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, b
         local += (clamp_len(T, p.T_cap) + TILE - 1) / TILE;
     }
     if (bad && report) set_status(p.status, STATUS_SEQLEN);
-    scratch[tid] = local;
+    // exclusive block scan of `local`: warp scans, then a scan of the warp totals
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) scratch[wid] = incl;
     __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int i = 0; i < nt; ++i) {
-            const int v = scratch[i];
-            scratch[i] = run;
-            run += v;
+    if (wid == 0) {
+        const int nw = nt >> 5;
+        int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += v;
         }
-        cu[p.B] = run * p.G;
+        if (lane < nw) scratch[lane] = w;  // inclusive prefix of warp totals
+        if (lane == nw - 1) cu[p.B] = w * p.G;
     }
     __syncthreads();
-    int run = scratch[tid];
+    int run = incl - local + (wid > 0 ? scratch[wid - 1] : 0);
     for (int b = b0; b < b1; ++b) {
         cu[b] = run * p.G;
         run += (clamp_len(p.seqlens[b], p.T_cap) + TILE - 1) / TILE;
@@ -146,7 +159,7 @@ __device__ __forceinline__ uint32_t swz(int tok, int dim) {
 // ----------------------------------------------------------------- bf16
 
 template <int D, int NMT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_split_bf16(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
     constexpr int HALVES = D / 64;
@@ -356,13 +369,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 {
                     const int tok = row0 + (((lane >> 3) & 1) << 3) + (lane & 7);
                     const int dsel = (lane >> 4) << 3;
+                    if (!split_p) {
 #pragma unroll
-                    for (int n2 = 0; n2 < D / 16; ++n2) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4_t(vbase + swz(tok, n2 * 16 + dsel), b0, b1, b2, b3);
-                        mma_16816(o[2 * n2], pa, b0, b1);
-                        mma_16816(o[2 * n2 + 1], pa, b2, b3);
-                        if (split_p) {
+                        for (int n2 = 0; n2 < D / 16; ++n2) {
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4_t(vbase + swz(tok, n2 * 16 + dsel), b0, b1, b2, b3);
+                            mma_16816(o[2 * n2], pa, b0, b1);
+                            mma_16816(o[2 * n2 + 1], pa, b2, b3);
+                        }
+                    } else {
+#pragma unroll
+                        for (int n2 = 0; n2 < D / 16; ++n2) {
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4_t(vbase + swz(tok, n2 * 16 + dsel), b0, b1, b2, b3);
+                            mma_16816(o[2 * n2], pa, b0, b1);
+                            mma_16816(o[2 * n2 + 1], pa, b2, b3);
                             mma_16816(o[2 * n2], pl, b0, b1);
                             mma_16816(o[2 * n2 + 1], pl, b2, b3);
                         }
@@ -562,30 +583,34 @@ __global__ void __launch_bounds__(128) decode_combine(const DecodeParams p, int 
         const long long s0 = cu[b] + (long long)g * ntb, s1 = s0 + ntb;
         const int c_lo = (int)(((s0 + 1) * C - 1) / W);
         const int c_hi = (int)((s1 * C - 1) / W);
-        // CTAs whose share is empty (more CTAs than tiles) wrote no record
+        // CTAs whose share is empty (more CTAs than tiles) wrote no record.
+        // One pass: running maximum, with the partial sums rescaled as it grows.
         auto empty_share = [&](int c) { return (long long)c * W / C == (long long)(c + 1) * W / C; };
-        float M = -INFINITY;
-        for (int c = c_lo; c <= c_hi; ++c)
-            if (!empty_share(c)) M = fmaxf(M, p.ws_ml[((long long)c + bg) * p.r + hl].x);
-        float L = 0.f;
+        float M = -INFINITY, L = 0.f;
+#pragma unroll 4
         for (int c = c_lo; c <= c_hi; ++c) {
             if (empty_share(c)) continue;
             const long long rec = (long long)c + bg;
             const float2 ml = p.ws_ml[rec * p.r + hl];
-            const float w = fast_exp2(ml.x - M);
-            L += w * ml.y;
             const float *src = p.ws_o + (rec * p.r + hl) * D + lane * PER;
+            float v[PER];
             if constexpr (PER == 4) {
-                const float4 v = *reinterpret_cast<const float4 *>(src);
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
-                acc[2] += w * v.z;
-                acc[3] += w * v.w;
+                const float4 t = *reinterpret_cast<const float4 *>(src);
+                v[0] = t.x;
+                v[1] = t.y;
+                v[2] = t.z;
+                v[3] = t.w;
             } else {
-                const float2 v = *reinterpret_cast<const float2 *>(src);
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
+                const float2 t = *reinterpret_cast<const float2 *>(src);
+                v[0] = t.x;
+                v[1] = t.y;
             }
+            const float Mn = fmaxf(M, ml.x);
+            const float a = fast_exp2(M - Mn), w = fast_exp2(ml.x - Mn);
+            L = L * a + w * ml.y;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) acc[k] = acc[k] * a + w * v[k];
+            M = Mn;
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
@@ -609,18 +634,42 @@ __global__ void __launch_bounds__(128) decode_combine(const DecodeParams p, int 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Raises a kernel's dynamic shared-memory limit once per device (the
+// attribute persists); one instance per kernel through the Tag parameter.
+template <typename Tag, typename Kern>
+cudaError_t set_smem_once(Kern kern, size_t smem) {
+    static std::atomic<int> done[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = dev >= 0 && dev < 64;
+    if (cached && done[dev].load(std::memory_order_acquire) >= (int)smem) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess && cached) {
+        int cur = done[dev].load();
+        while (cur < (int)smem && !done[dev].compare_exchange_weak(cur, (int)smem)) {
+        }
+    }
+    return e;
+}
+
+template <int D, int NMT>
+struct Bf16Tag {};
+template <int D>
+struct F32Tag {};
+
 int bf16_nmt(int r) { return r <= 16 ? 1 : (r <= 32 ? 2 : 4); }
 
 size_t smem_bf16(int D, int nmt, int B) {
     const int nsl = kCWarps / nmt;
     const size_t red = nsl > 1 ? (size_t)nsl * nmt * 16 * (D + 2) * 4 : 0;
     return 1024 + (size_t)kStages * 2 * kTile * D * 2 + red + 2 * kStages * 8 + 4 +
-           (size_t)(B + 1) * 4 + kThreads * 4;
+           (size_t)(B + 1) * 4 + 32 * 4;
 }
 
 size_t smem_f32(int D, int r, int B) {
     return ((size_t)2 * kTileF32 * (D + 1) + 4 * 32 + 2 * (size_t)r * D + 2 * r) * 4 +
-           (size_t)(B + 1) * 4 + kThreadsF32 * 4;
+           (size_t)(B + 1) * 4 + 32 * 4;
 }
 
 template <int D, int NMT>
@@ -628,7 +677,7 @@ cudaError_t run_bf16(const DecodeParams &p, const CUtensorMap *tmk, const CUtens
                      int ctas, cudaStream_t st) {
     const size_t smem = smem_bf16(D, NMT, p.B);
     auto kern = decode_split_bf16<D, NMT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once<Bf16Tag<D, NMT>>(kern, smem);
     if (e != cudaSuccess) return e;
     kern<<<ctas, kThreads, smem, st>>>(*tmk, *tmv, p);
     return cudaGetLastError();
@@ -638,7 +687,7 @@ template <int D>
 cudaError_t run_f32(const DecodeParams &p, int ctas, cudaStream_t st) {
     const size_t smem = smem_f32(D, p.r, p.B);
     auto kern = decode_split_f32<D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once<F32Tag<D>>(kern, smem);
     if (e != cudaSuccess) return e;
     kern<<<ctas, kThreadsF32, smem, st>>>(p);
     return cudaGetLastError();
@@ -667,7 +716,8 @@ DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, i
     const int r = H / G;
     const int tile = dtype == GQA_BF16 ? kTile : kTileF32;
     const long long max_tiles = (long long)B * G * ((T_cap + tile - 1) / tile);
-    long long ctas = force_ctas > 0 ? force_ctas : (long long)num_sms;
+    long long ctas = force_ctas > 0 ? force_ctas
+                                    : (long long)num_sms * (dtype == GQA_BF16 ? kCtasPerSm : 1);
     if (ctas > max_tiles) ctas = max_tiles;
     if (ctas < 1) ctas = 1;
     L.ctas = (int)ctas;
