@@ -90,7 +90,8 @@ def max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -231,8 +232,8 @@ class Decode:
         order = torch.randperm(rows_total, generator=gen).tolist()
         k_host = x.k_cache if x.k_cache.device.type == "cpu" else None
         done, t_used, tokens = 0, 0.0, 0
-        n = 8
-        while done < rows_total and t_used < budget_s:
+        n = 1
+        while done < rows_total and (done == 0 or t_used < budget_s):
             rows = order[done:done + n]
             if k_host is None:   # device-drawn cache: copy the slabs of one sequence
                 b = rows[0] // x.H
@@ -247,7 +248,7 @@ class Decode:
             t_used += time.perf_counter() - t0
             tokens += sum(int(x.seqlens[r // x.H].clamp(0, x.T_cap)) for r in rows)
             done += len(rows)
-            n = min(4 * n, 512)
+            n = min(2 * n, 512)
         # tokens here are (query head, key) pairs; convert to the step's KV bytes
         frac = tokens / (self.sum_T * x.H)
         return {"seconds": t_used, "fraction_of_step": frac,
@@ -294,8 +295,8 @@ class Prefill:
         gen = torch.Generator().manual_seed(7)
         total = x.B * x.S * x.H
         done, t_used, flops = 0, 0.0, 0
-        n = 16
-        while t_used < budget_s and done < total:
+        n = 1
+        while done < total and (done == 0 or t_used < budget_s):
             rows = torch.randint(0, total, (n,), generator=gen).tolist()
             t0 = time.perf_counter()
             oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, rows=rows)
@@ -439,7 +440,8 @@ def run_reference(args, world, rank):
 
     name = args.workload or HEADLINE
     wl = make_host_only(name)
-    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    # the whole reference run stays within about a minute and a half of oracle time
+    per_step = min(2.0, 90.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         wl.oracle_sample(per_step / 4)
     secs, frac = 0.0, 0.0
