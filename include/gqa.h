@@ -150,7 +150,7 @@ GQA_API int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v
  *   q    device, [B, S, H, d_h] bf16, 16-byte aligned
  *   k, v device, [B, S, G, d_h] bf16, 16-byte aligned
  *   out  device, [B, S, H, d_h] bf16, 16-byte aligned
- *   Supported: dt = GQA_BF16, d_h = 128, H/G even; any S >= 1.
+ *   Supported: dt = GQA_BF16, d_h = 128, H/G even, scale > 0; any S >= 1.
  * Internally: tcgen05 tensor-core MMAs with fp32 accumulators in tensor
  * memory, TMA-fed shared-memory tiles, fp32 online softmax, P in bf16.
  */

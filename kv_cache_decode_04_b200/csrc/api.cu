@@ -227,7 +227,8 @@ int gqa_prefill_causal(const void *q, const void *k, const void *v, void *out, i
     if (rc) return rc;
     if (S <= 0) return fail(GQA_ERR_INVALID, "S must be positive");
     if (!q || !k || !v || !out) return fail(GQA_ERR_INVALID, "null tensor pointer");
-    if (!std::isfinite(scale)) return fail(GQA_ERR_INVALID, "scale must be finite");
+    if (!std::isfinite(scale) || !(scale > 0.f))
+        return fail(GQA_ERR_INVALID, "prefill scale must be finite and positive");
     if (dt != GQA_BF16) return fail(GQA_ERR_UNSUPPORTED, "prefill supports bf16 only");
     if (d_h != 128) return fail(GQA_ERR_UNSUPPORTED, "prefill supports d_h=128 only (got %d)", d_h);
     if ((H / G) % 2 != 0) return fail(GQA_ERR_UNSUPPORTED, "prefill needs an even H/G (got %d)", H / G);

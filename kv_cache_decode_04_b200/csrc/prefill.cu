@@ -26,6 +26,7 @@
 // Only KV tiles j <= query tile are visited; the diagonal tile is masked
 // (key > query -> -inf).
 #include "common.cuh"
+#include "exp2_fma.cuh"
 #include "gqa.h"
 #include "internal.h"
 #include "tc.cuh"
@@ -45,8 +46,8 @@ constexpr int kThreads = 384;           // 3 warpgroups
 // 384*kLaunchRegs, or an .inc would wait for registers that never come; the
 // launcher checks the compiled register count against this before launching.
 constexpr int kLaunchRegs = 168;
-constexpr int kLowRegs = 88;
-constexpr int kHighRegs = 208;
+constexpr int kLowRegs = 136;
+constexpr int kHighRegs = 184;
 static_assert(2 * 128 * kHighRegs + 128 * kLowRegs <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kOffQ = 0;                 // Q0, Q1
@@ -71,6 +72,26 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, uint64_
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w),
         "l"(policy)
         : "memory");
+}
+
+// Packed pairs of fp32 (Blackwell's paired FMA/ADD datapath).
+__device__ __forceinline__ uint64_t f32x2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
 }
 
 // Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
@@ -280,16 +301,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, sr[c]);
             tc::wait_ld();
             const bool diag = (j == n_kv - 1);
-            float mx = -INFINITY;
+            if (diag) {  // keys after the query row are masked
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (c * 32 + e > t) sr[c][e] = __float_as_uint(-INFINITY);
+            }
+            // Row maximum of the raw scores (the scale is positive), with eight
+            // independent partial maxima instead of one 128-long chain.
+            float mx8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float x = __uint_as_float(sr[c][e]) * p.scale_log2;
-                    if (diag && (c * 32 + e) > t) x = -INFINITY;
-                    sr[c][e] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
-                }
+                for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[c][e]));
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
             float alpha = 1.f;
             bool rescale = false;
             if (j == 0) {
@@ -304,20 +333,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l *= alpha;
                 }
             }
-            // P = 2^(x - m) in bf16 pairs over the first 64 columns of this S block.
+            // P = 2^(s * scale_log2 - m) in bf16 pairs over the first 64 columns of
+            // this S block; the exponent argument is formed two at a time (packed
+            // fp32 FMA) and the row sum kept in four packed partial sums.
             // Rows of the first query tile see at most 128 keys, too few for the bf16
             // rounding of P to average out; there P is carried as P_hi + P_lo (two bf16
             // terms, about 16 significant bits), P_lo in columns 64..127.
-            float rs = 0.f;
-            if (!split_p) {
+            const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2);
+            const uint64_t nm2 = f32x2_pack(-m, -m);
+            uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+            if (!split_p && !diag) {
+                // Off-diagonal tiles: one exponential in four on the FMA pipe
+                // (exp2_fma), the rest on the special-function unit.
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = fast_exp2(__uint_as_float(sr[c4][2 * e]) - m);
-                        const float p1 = fast_exp2(__uint_as_float(sr[c4][2 * e + 1]) - m);
-                        rs += p0 + p1;
+                        float x0, x1;
+                        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sr[c4][2 * e]),
+                                                          __uint_as_float(sr[c4][2 * e + 1])), sc2, nm2), x0, x1);
+                        const float p0 = (e & 3) == 3 ? exp2_fma(x0) : fast_exp2(x0);
+                        const float p1 = (e & 3) == 3 ? exp2_fma(x1) : fast_exp2(x1);
+                        rs2[e & 3] = f32x2_add(rs2[e & 3], f32x2_pack(p0, p1));
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tc::st16(tS + c4 * 16, pk);
+                }
+            } else if (!split_p) {
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float x0, x1;
+                        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sr[c4][2 * e]),
+                                                          __uint_as_float(sr[c4][2 * e + 1])), sc2, nm2), x0, x1);
+                        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                        rs2[e & 3] = f32x2_add(rs2[e & 3], f32x2_pack(p0, p1));
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                     tc::st16(tS + c4 * 16, pk);
@@ -331,9 +384,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int e1 = 0; e1 < 4; ++e1) {
                             const int e = e4 * 4 + e1;
-                            const float p0 = fast_exp2(__uint_as_float(sr[c4][2 * e]) - m);
-                            const float p1 = fast_exp2(__uint_as_float(sr[c4][2 * e + 1]) - m);
-                            rs += p0 + p1;
+                            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e]), p.scale_log2, -m));
+                            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e + 1]), p.scale_log2, -m));
+                            rs2[e1] = f32x2_add(rs2[e1], f32x2_pack(p0, p1));
                             ph[e1] = pack_bf16x2(p0, p1);
                             const float2 h = unpack_bf16x2(ph[e1]);
                             pl[e1] = pack_bf16x2(p0 - h.x, p1 - h.y);
@@ -342,6 +395,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::st4(tS + 64 + c4 * 16 + e4 * 4, pl);
                     }
                 }
+            }
+            float rs = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float a0, a1;
+                f32x2_unpack(rs2[i], a0, a1);
+                rs += a0 + a1;
             }
             if (rescale) {  // O was last written by the P.V of tile j-1, complete by now
 #pragma unroll 1
