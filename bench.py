@@ -37,7 +37,8 @@ import gqa_inputs as gi  # noqa: E402
 METRIC = "GQA decode achieved HBM GB/s (% of peak) & attn-tokens/s; prefill TFLOP/s"
 HEADLINE = "llama2_7b_decode"
 ROW_WORKLOADS = ["tiny_decode_fp32", "llama2_70b_ragged_decode"] + \
-    ["long_ctx_decode_G%d" % g for g in (1, 2, 4, 8, 16, 32)] + ["causal_prefill", "meanpool_init"]
+    ["long_ctx_decode_G%d" % g for g in (1, 2, 4, 8, 16, 32)] + ["causal_prefill", "meanpool_init",
+                                                                "qkv_append_llama2_7b"]
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, bytes, from ncu
 # captures of the current kernels (profiles/*.md); a workload missing here has
@@ -349,9 +350,57 @@ class MeanPool:
                 "sample": "the whole conversion (both W_K and W_V)"}
 
 
+class QkvAppend:
+    """One decode token's Q/K/V projections with the KV-cache append."""
+    kind = "qkv"
+
+    def __init__(self, name, gqa, device="cuda"):
+        w = gi.WORKLOADS[name]
+        self.name, self.w, self.gqa = name, w, gqa
+        x = gi.qkv_inputs(w["B"], w["d"], w["H"], w["G"], w["d_h"], w["T"], w["dtype"], seed=0)
+        self.x = x
+        self.h, self.wq, self.wk, self.wv = (t.to(device) for t in (x.h, x.W_Q, x.W_K, x.W_V))
+        self.kc, self.vc = x.k_cache.to(device), x.v_cache.to(device)
+        self.sl = x.seqlens.to(device)
+        self.q = torch.empty((x.B, x.H, x.d_h), dtype=x.h.dtype, device=device)
+        self.sl_out = torch.empty_like(self.sl)
+        e = x.h.element_size()
+        # weights read once, h read, q written, one k and one v row per KV head written
+        self.bytes = (x.d * (x.H + 2 * x.G) * x.d_h + x.B * x.d + x.B * x.H * x.d_h
+                      + 2 * x.B * x.G * x.d_h) * e
+        self.launches_per_step = (x.B + 31) // 32
+        self.dtype = "bf16"
+
+    def step(self, stream=None):
+        self.gqa.qkv_append(self.h, self.wq, self.wk, self.wv, self.kc, self.vc, self.sl,
+                            q_out=self.q, seqlens_out=self.sl_out, stream=stream)
+
+    def config(self):
+        x = self.x
+        return {"workload": self.name, "B": x.B, "d": x.d, "H": x.H, "G": x.G, "d_h": x.d_h,
+                "T_cap": x.T_cap}
+
+    def metric(self, sps, n_ranks):
+        return {"value": n_ranks * self.bytes / sps / 1e9, "unit": "GB/s"}
+
+    def roofline(self, sps, peaks, which, long_run=False):
+        a = self.bytes / sps / 1e9
+        return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": a / peaks["hbm_gbs"], "peak_source": which + " hbm_gbs",
+                "traffic": NCU_TRAFFIC.get(self.name)}
+
+    def oracle_sample(self, budget_s):
+        import oracle
+        x = self.x
+        t0 = time.perf_counter()
+        oracle.qkv_append(x.h[:1], x.W_Q, x.W_K, x.W_V, x.k_cache[:1], x.v_cache[:1], x.seqlens[:1])
+        return {"seconds": time.perf_counter() - t0, "fraction_of_step": 1.0 / x.B,
+                "sample": "the projections and append of sequence 0 of %d" % x.B}
+
+
 def make(name, gqa):
     kind = gi.WORKLOADS[name]["kind"]
-    return {"decode": Decode, "prefill": Prefill, "meanpool": MeanPool}[kind](name, gqa)
+    return {"decode": Decode, "prefill": Prefill, "meanpool": MeanPool, "qkv": QkvAppend}[kind](name, gqa)
 
 
 # ------------------------------------------------------------------ timing

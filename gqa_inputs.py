@@ -29,6 +29,9 @@ WORKLOADS = {
                            dtype=torch.bfloat16),
     "meanpool_init": dict(kind="meanpool", H=64, G=8, d_h=128, d=8192,
                           dtype=torch.bfloat16, std=0.02),
+    # one decode token's projections + cache append, Llama-2-7B shape (d = 4096)
+    "qkv_append_llama2_7b": dict(kind="qkv", B=16, d=4096, H=32, G=8, d_h=128, T=4096,
+                                 dtype=torch.bfloat16),
     # half-length prefill (150 MB of q/k/v/out, above the 126 MB L2) for profiler captures
     "causal_prefill_profile": dict(kind="prefill", B=1, S=4096, H=64, G=8, d_h=128,
                                    dtype=torch.bfloat16),
@@ -130,6 +133,42 @@ def meanpool_inputs(H, d_h, d, dtype=torch.bfloat16, seed=0, std=0.02):
     return wk, wv
 
 
+@dataclass
+class QkvInputs:
+    h: torch.Tensor
+    W_Q: torch.Tensor
+    W_K: torch.Tensor
+    W_V: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    seqlens: torch.Tensor
+    B: int
+    d: int
+    H: int
+    G: int
+    d_h: int
+    T_cap: int
+
+
+def qkv_inputs(B, d, H, G, d_h, T_cap, dtype=torch.bfloat16, seed=0, seqlens=None):
+    """h [B, d] ~ N(0, 1); W_Q [d, H*d_h], W_K/W_V [d, G*d_h] ~ N(0, d^-1/2) (so the
+    projections are O(1)); caches [B, G, T_cap, d_h] ~ N(0, 1); seqlens default
+    T_cap - 1 (one free slot).  Draw order: h, W_Q, W_K, W_V, K cache, V cache."""
+    gen = torch.Generator().manual_seed(seed)
+    h = _randn((B, d), gen, dtype)
+    w_std = d ** -0.5
+    wq = _randn((d, H * d_h), gen, dtype, w_std)
+    wk = _randn((d, G * d_h), gen, dtype, w_std)
+    wv = _randn((d, G * d_h), gen, dtype, w_std)
+    kc = _randn((B, G, T_cap, d_h), gen, dtype)
+    vc = _randn((B, G, T_cap, d_h), gen, dtype)
+    if seqlens is None:
+        sl = torch.full((B,), T_cap - 1, dtype=torch.int32)
+    else:
+        sl = torch.as_tensor(seqlens, dtype=torch.int32).reshape(B)
+    return QkvInputs(h, wq, wk, wv, kc, vc, sl, B, d, H, G, d_h, T_cap)
+
+
 def workload_inputs(name, seed=0):
     w = WORKLOADS[name]
     if w["kind"] == "decode":
@@ -137,4 +176,6 @@ def workload_inputs(name, seed=0):
                              ragged=w["ragged"])
     if w["kind"] == "prefill":
         return prefill_inputs(w["B"], w["S"], w["H"], w["G"], w["d_h"], w["dtype"], seed)
+    if w["kind"] == "qkv":
+        return qkv_inputs(w["B"], w["d"], w["H"], w["G"], w["d_h"], w["T"], w["dtype"], seed)
     return meanpool_inputs(w["H"], w["d_h"], w["d"], w["dtype"], seed, w["std"])

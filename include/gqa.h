@@ -176,6 +176,36 @@ GQA_API int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *
                     gqa_stream_t stream);
 
 /*
+ * gqa_qkv_append -- the step before decode, fused: one new token's query,
+ * key and value projections, with the key and value written straight into
+ * the KV cache ("Grouped-Query Attention", llm-arch-kb, section 3
+ * "Reference implementation": q = h W_Q, k = h W_K, v = h W_V with only G
+ * key/value heads; section 1 "Premise": the cache grows by one key and one
+ * value vector per token, head and layer):
+ *     q_out[b]               = h[b] W_Q                      (H heads of d_h)
+ *     k_cache[b, g, T_b, :]  = (h[b] W_K)[g d_h : (g+1) d_h]  for each of G heads
+ *     v_cache[b, g, T_b, :]  = (h[b] W_V)[g d_h : (g+1) d_h]
+ *     seqlens_out[b]         = T_b + 1,     T_b = seqlens[b].
+ * bf16 inputs, fp32 accumulation, each output rounded once to bf16.  Cache
+ * positions other than T_b are not touched.  A sequence whose cache is full
+ * (T_b >= T_cap) or whose T_b is negative gets no append, keeps
+ * seqlens_out[b] = T_b and flags GQA_ERR_SEQLEN.
+ *
+ *   h                 device, [B, d] bf16, 16-byte aligned
+ *   W_Q               device, [d, H*d_h] bf16 row-major, 16-byte aligned
+ *   W_K, W_V          device, [d, G*d_h] bf16 row-major, 16-byte aligned
+ *   q_out             device, [B, H, d_h] bf16
+ *   k_cache, v_cache  device, [B, G, T_cap, d_h] bf16 (updated in place)
+ *   seqlens           device, [B] int32 (read only)
+ *   seqlens_out       device, [B] int32, or NULL; must not overlap seqlens
+ *   Supported: dt = GQA_BF16, d a multiple of 128, d_h in {64, 128}.
+ */
+GQA_API int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V,
+                           void *q_out, void *k_cache, void *v_cache, const int32_t *seqlens,
+                           int32_t *seqlens_out, int B, int d, int H, int G, int d_h, int T_cap,
+                           gqa_dtype dt, gqa_stream_t stream);
+
+/*
  * gqa_get_status -- synchronises `stream`, then reads and clears the device
  * status word: GQA_OK, GQA_ERR_SEQLEN or GQA_ERR_TIMEOUT (device-side
  * conditions of earlier calls on this device), or GQA_ERR_CUDA if the

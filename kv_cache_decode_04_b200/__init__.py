@@ -23,6 +23,7 @@ import os
 import torch
 
 __all__ = ["decode", "decode_noalloc", "decode_workspace_bytes", "prefill_causal", "meanpool_kv",
+           "qkv_append",
            "kv_cache_bytes", "get_status", "GQAError", "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqa.so")
@@ -33,8 +34,8 @@ _ERRORS = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGN", -4: "CUDA", -5: "WORKS
 
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_kv_cache_bytes", "gqa_decode_workspace_bytes", "gqa_decode",
-           "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_status",
-           "gqa_last_error_string", "gqa_version")
+           "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_qkv_append",
+           "gqa_get_status", "gqa_last_error_string", "gqa_version")
 
 
 class GQAError(RuntimeError):
@@ -61,6 +62,9 @@ def _load():
     L.gqa_prefill_causal.restype = i32
     L.gqa_meanpool_kv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     L.gqa_meanpool_kv.restype = i32
+    L.gqa_qkv_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                 i32, vp]
+    L.gqa_qkv_append.restype = i32
     L.gqa_get_status.argtypes = [vp]
     L.gqa_get_status.restype = i32
     L.gqa_last_error_string.argtypes = []
@@ -198,6 +202,33 @@ def meanpool_kv(wk, wv, G, out_k=None, out_v=None, stream=None):
                              _dev(out_v, "WV_out"), H, int(G), d_h, d, code, _stream(stream))
     _check(rc)
     return out_k, out_v
+
+
+def qkv_append(h, W_Q, W_K, W_V, k_cache, v_cache, seqlens, q_out=None, seqlens_out=None,
+               stream=None):
+    """One decode token: q = h W_Q, and h W_K, h W_V appended to the KV cache.
+
+    h [B, d]; W_Q [d, H*d_h]; W_K, W_V [d, G*d_h]; k_cache, v_cache
+    [B, G, T_cap, d_h] (written in place at position seqlens[b]); seqlens [B]
+    int32.  Returns (q_out [B, H, d_h], seqlens_out [B] = seqlens + 1).
+    """
+    B, d = h.shape
+    _, G, T_cap, d_h = k_cache.shape
+    H = W_Q.shape[1] // d_h
+    if tuple(W_Q.shape) != (d, H * d_h) or tuple(W_K.shape) != (d, G * d_h) or \
+            tuple(W_V.shape) != (d, G * d_h) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between h, the weights and the caches")
+    code = _dtype_code(h)
+    if q_out is None:
+        q_out = torch.empty((B, H, d_h), dtype=h.dtype, device=h.device)
+    if seqlens_out is None:
+        seqlens_out = torch.empty_like(seqlens)
+    rc = lib.gqa_qkv_append(_dev(h, "h"), _dev(W_Q, "W_Q"), _dev(W_K, "W_K"), _dev(W_V, "W_V"),
+                            _dev(q_out, "q_out"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                            _dev(seqlens, "seqlens"), _dev(seqlens_out, "seqlens_out"), B, d, H, G,
+                            d_h, T_cap, code, _stream(stream))
+    _check(rc)
+    return q_out, seqlens_out
 
 
 def get_status(stream=None):

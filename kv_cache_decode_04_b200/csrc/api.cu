@@ -309,6 +309,73 @@ int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *WV_out, 
     return GQA_OK;
 }
 
+int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V, void *q_out,
+                   void *k_cache, void *v_cache, const int32_t *seqlens, int32_t *seqlens_out, int B, int d,
+                   int H, int G, int d_h, int T_cap, gqa_dtype dt, gqa_stream_t stream) {
+    t_err[0] = 0;
+    int rc = check_dims(B, H, G, d_h);
+    if (rc) return rc;
+    if (d <= 0 || T_cap <= 0) return fail(GQA_ERR_INVALID, "d and T_cap must be positive");
+    if (!h || !W_Q || !W_K || !W_V || !q_out || !k_cache || !v_cache || !seqlens)
+        return fail(GQA_ERR_INVALID, "null tensor pointer");
+    if (dt != GQA_BF16) return fail(GQA_ERR_UNSUPPORTED, "qkv_append supports bf16 only");
+    if (d_h != 64 && d_h != 128) return fail(GQA_ERR_UNSUPPORTED, "d_h=%d (built: 64, 128)", d_h);
+    if (d % 128 != 0) return fail(GQA_ERR_UNSUPPORTED, "d=%d must be a multiple of 128", d);
+    if (seqlens_out && seqlens_out < seqlens + B && seqlens < seqlens_out + B)
+        return fail(GQA_ERR_INVALID, "seqlens_out must not overlap seqlens");
+    if ((long long)B * G * T_cap * d_h >= (1ll << 40)) return fail(GQA_ERR_UNSUPPORTED, "cache too large");
+    if (misaligned(W_Q, 16) || misaligned(W_K, 16) || misaligned(W_V, 16) || misaligned(h, 16) ||
+        misaligned(q_out, 2) || misaligned(k_cache, 2) || misaligned(v_cache, 2) || misaligned(seqlens, 4) ||
+        misaligned(seqlens_out, 4))
+        return fail(GQA_ERR_ALIGN, "weights and h must be 16-byte aligned");
+    DeviceInfo *dev = nullptr;
+    rc = device_info(&dev);
+    if (rc) return rc;
+    CUtensorMap tq, tk, tv;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)H * d_h, (cuuint64_t)d};
+        const cuuint64_t strides[1] = {(cuuint64_t)H * d_h * 2};
+        const cuuint32_t box[2] = {64, 128};
+        rc = make_tmap_bf16(&tq, W_Q, 2, dims, strides, box);
+        if (rc) return rc;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)G * d_h, (cuuint64_t)d};
+        const cuuint64_t strides[1] = {(cuuint64_t)G * d_h * 2};
+        const cuuint32_t box[2] = {64, 128};
+        rc = make_tmap_bf16(&tk, W_K, 2, dims, strides, box);
+        if (rc) return rc;
+        rc = make_tmap_bf16(&tv, W_V, 2, dims, strides, box);
+        if (rc) return rc;
+    }
+    CUtensorMap th;  // h [B, d]: boxes of 32 sequences x 64 features (rows past B read as 0)
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)B};
+        const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+        const cuuint32_t box[2] = {64, 32};
+        rc = make_tmap_bf16(&th, h, 2, dims, strides, box);
+        if (rc) return rc;
+    }
+    gqa::QkvArgs a = {};
+    a.h = h;
+    a.q_out = q_out;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.seqlens = seqlens;
+    a.seqlens_out = seqlens_out;
+    a.B = B;
+    a.d = d;
+    a.H = H;
+    a.G = G;
+    a.d_h = d_h;
+    a.T_cap = T_cap;
+    a.status = dev->status;
+    a.timeout_ns = wait_timeout_ns();
+    cudaError_t e = gqa::launch_qkv_append(a, &tq, &tk, &tv, &th, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "qkv_append launch");
+    return GQA_OK;
+}
+
 int gqa_get_status(gqa_stream_t stream) {
     t_err[0] = 0;
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

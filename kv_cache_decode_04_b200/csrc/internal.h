@@ -54,6 +54,19 @@ struct PrefillArgs {
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const CUtensorMap *tmk,
                            const CUtensorMap *tmv, cudaStream_t stream);
 
+// One decode token's Q/K/V projections and the KV-cache append.
+struct QkvArgs {
+    const void *h;
+    void *q_out, *k_cache, *v_cache;
+    const int32_t *seqlens;
+    int32_t *seqlens_out;
+    int B, d, H, G, d_h, T_cap;
+    unsigned *status;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUtensorMap *tk,
+                              const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t stream);
+
 // Records `msg` as the calling thread's last error and returns `code`.
 int set_error(int code, const char *msg);
 

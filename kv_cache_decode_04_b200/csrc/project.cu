@@ -1,0 +1,253 @@
+// project.cu -- one decode token's Q/K/V projections and the KV-cache append.
+//
+// What is computed ("Grouped-Query Attention", llm-arch-kb, section 3
+// "Reference implementation": q = h W_Q, k = h W_K, v = h W_V with W_Q
+// [d, H d_h] and W_K, W_V [d, G d_h]; section 1 "Premise": the cache grows by
+// one key and one value vector per token, head and layer):
+//     q[b]                     = h[b] W_Q                 -> q_out [B, H, d_h]
+//     k_cache[b, g, T_b, :]    = (h[b] W_K)[g*d_h : (g+1)*d_h]
+//     v_cache[b, g, T_b, :]    = (h[b] W_V)[g*d_h : (g+1)*d_h]
+//     seqlens_out[b]           = T_b + 1,   with T_b = seqlens[b].
+// The K/V projection is G/H the size of the Q one: the "GEMM shrink" of
+// section 2 ("at decode the GEMM and the cache read both shrink by H/G").
+//
+// This is a skinny GEMM (B rows) bound by reading the weights once.  One CTA
+// owns 64 output columns of one of the three weights and streams them in
+// [128 rows x 64 columns] TMA tiles (128-byte swizzle) through a 6-stage
+// ring, together with the matching [32 sequences x 128] slice of h; four
+// warps split each tile's sixteen-row K-steps and run warp-level bf16 MMAs (B
+// padded to 16-row blocks), then the four partial sums are added in a fixed
+// order in shared memory, rounded once to bf16 and written.
+#include "common.cuh"
+#include "gqa.h"
+#include "internal.h"
+
+namespace gqa {
+
+namespace {
+
+constexpr int kNT = 64;                    // output columns per CTA
+constexpr int kKT = 128;                   // weight rows per stage
+constexpr int kStagesP = 6;
+constexpr int kCW = 4;                     // MMA warps
+constexpr int kThreadsP = (kCW + 1) * 32;  // + 1 TMA warp
+constexpr int kTileB = kKT * kNT * 2;      // 16 KB of weights per stage
+constexpr int kHRows = 32;                 // sequences per launch (h box height)
+constexpr int kHHalf = kHRows * 128;       // one [32 x 64] bf16 box of h, 4 KB
+constexpr int kStageB = kTileB + 2 * kHHalf;
+
+struct ProjParams {
+    const __nv_bfloat16 *h;   // [B, d]
+    __nv_bfloat16 *q_out;     // [B, H*d_h]
+    __nv_bfloat16 *k_cache;   // [B, G, T_cap, d_h]
+    __nv_bfloat16 *v_cache;
+    const int32_t *seqlens;
+    int32_t *seqlens_out;     // may be null
+    unsigned *status;
+    int B, d, H, G, d_h, T_cap;
+    int b0;                   // first sequence of this launch
+    int nq, nk;               // 64-column blocks of W_Q and of W_K (= of W_V)
+    unsigned long long timeout_ns;
+};
+
+// [128 rows x 64 bf16] tile, 128-byte swizzle: 16-byte chunk ^= row mod 8.
+__device__ __forceinline__ uint32_t swz64(int row, int col) {
+    return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + ((col & 7) << 1));
+}
+
+template <int RB>  // 16-row blocks of sequences in this launch (1 or 2)
+__global__ void __launch_bounds__(kThreadsP, 1)
+    qkv_append_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmh,
+                      const ProjParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    float *red = reinterpret_cast<float *>(sm + kStagesP * kStageB);  // [kCW][RB*16][kNT]
+    uint64_t *full = reinterpret_cast<uint64_t *>(red + kCW * RB * 16 * kNT);
+    uint64_t *empty = full + kStagesP;
+    int *abort_flag = reinterpret_cast<int *>(empty + kStagesP);
+    volatile int *vabort = abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cb = blockIdx.x;
+    const int region = cb < p.nq ? 0 : (cb < p.nq + p.nk ? 1 : 2);  // Q, K, V
+    const int col0 = (cb - (region == 0 ? 0 : (region == 1 ? p.nq : p.nq + p.nk))) * kNT;
+    const CUtensorMap *tm = region == 0 ? &tmq : (region == 1 ? &tmk : &tmv);
+    const int n_kt = p.d / kKT;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kCW);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == kCW) {  // ---------------- TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(tm);
+            tma_prefetch_desc(&tmh);
+            const uint64_t pol = l2_policy_evict_first();
+            const uint64_t pol_h = l2_policy_evict_last();  // h is read by every CTA
+            for (int kt = 0; kt < n_kt; ++kt) {
+                const int s = kt % kStagesP;
+                const uint32_t ph = (kt / kStagesP) & 1;
+                if (*vabort || !mbar_wait(&empty[s], ph ^ 1, p.timeout_ns)) {
+                    set_status(p.status, STATUS_TIMEOUT);
+                    *vabort = 1;
+                    break;
+                }
+                uint8_t *st = sm + s * kStageB;
+                mbar_arrive_expect_tx(&full[s], kStageB);
+                tma_load_2d(st, tm, &full[s], col0, kt * kKT, pol);
+                tma_load_2d(st + kTileB, &tmh, &full[s], kt * kKT, p.b0, pol_h);
+                tma_load_2d(st + kTileB + kHHalf, &tmh, &full[s], kt * kKT + 64, p.b0, pol_h);
+            }
+        }
+        return;
+    }
+
+    // ---------------- MMA warps: warp w takes K-steps 2w and 2w+1 of each tile
+    const int g8 = lane >> 2, q4 = lane & 3;
+    float acc[RB][8][4];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) acc[rb][nt][0] = acc[rb][nt][1] = acc[rb][nt][2] = acc[rb][nt][3] = 0.f;
+    bool dead = false;
+    for (int kt = 0; kt < n_kt; ++kt) {
+        const int s = kt % kStagesP;
+        const uint32_t ph = (kt / kStagesP) & 1;
+        if (!dead && (*vabort || !mbar_wait(&full[s], ph, p.timeout_ns))) {
+            dead = true;
+            *vabort = 1;
+            set_status(p.status, STATUS_TIMEOUT);
+        }
+        if (!dead) {
+            const uint32_t base = smem_u32(sm + s * kStageB);
+            const uint32_t hbase = base + kTileB;
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int ks = 2 * warp + k2;
+                // A fragments of h (rows = sequences, k contiguous) from the staged slice;
+                // sequences past B were zero-filled by the copy
+                uint32_t a[RB][4];
+                const int kc = ks * 16 + ((lane >> 4) << 3);  // k column in the 128-wide slice
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    const int hr = rb * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+                    ldsm_x4(hbase + (kc >> 6) * kHHalf + swz64(hr, kc & 63), a[rb][0], a[rb][1], a[rb][2],
+                            a[rb][3]);
+                }
+                const int row = ks * 16 + (((lane >> 3) & 1) << 3) + (lane & 7);
+#pragma unroll
+                for (int n2 = 0; n2 < 4; ++n2) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(base + swz64(row, n2 * 16 + ((lane >> 4) << 3)), b0, b1, b2, b3);
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb) {
+                        mma_16816(acc[rb][2 * n2], a[rb], b0, b1);
+                        mma_16816(acc[rb][2 * n2 + 1], a[rb], b2, b3);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // ---------------- fixed-order sum of the four K-slices, one rounding, write
+    float *my = red + warp * RB * 16 * kNT;
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            const int c = nt * 8 + 2 * q4;
+            my[(rb * 16 + g8) * kNT + c] = acc[rb][nt][0];
+            my[(rb * 16 + g8) * kNT + c + 1] = acc[rb][nt][1];
+            my[(rb * 16 + g8 + 8) * kNT + c] = acc[rb][nt][2];
+            my[(rb * 16 + g8 + 8) * kNT + c + 1] = acc[rb][nt][3];
+        }
+    asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
+    if (dead) return;
+    const int per = RB * 16 * kNT;
+    for (int idx = tid; idx < per; idx += kCW * 32) {
+        const int row = idx / kNT, c = idx - row * kNT;
+        const int b = p.b0 + row;
+        if (b >= p.B) continue;
+        float v = red[idx];
+#pragma unroll
+        for (int w = 1; w < kCW; ++w) v += red[w * per + idx];
+        const __nv_bfloat16 o = __float2bfloat16_rn(v);
+        const int n = col0 + c;
+        if (region == 0) {
+            p.q_out[(size_t)b * p.H * p.d_h + n] = o;
+        } else {
+            const int T = p.seqlens[b];
+            if (T < 0 || T >= p.T_cap) {
+                if (c == 0 && col0 == 0) set_status(p.status, STATUS_SEQLEN);  // full cache: no append
+                continue;
+            }
+            const int g = n / p.d_h, dim = n - g * p.d_h;
+            __nv_bfloat16 *cache = region == 1 ? p.k_cache : p.v_cache;
+            cache[(((size_t)b * p.G + g) * p.T_cap + T) * p.d_h + dim] = o;
+        }
+    }
+    if (cb == 0 && p.seqlens_out)
+        for (int b = p.b0 + tid; b < min(p.B, p.b0 + RB * 16); b += kCW * 32) {
+            const int T = p.seqlens[b];
+            p.seqlens_out[b] = (T >= 0 && T < p.T_cap) ? T + 1 : T;
+        }
+}
+
+template <int RB>
+cudaError_t run_proj(const ProjParams &p, const CUtensorMap *tq, const CUtensorMap *tk, const CUtensorMap *tv,
+                     const CUtensorMap *th, cudaStream_t st) {
+    const size_t smem = 1024 + (size_t)kStagesP * kStageB + (size_t)kCW * RB * 16 * kNT * 4 + 2 * kStagesP * 8 + 16;
+    static int set_for[64];  // largest shared-memory size set, per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || set_for[dev] < (int)smem) {
+        e = cudaFuncSetAttribute(qkv_append_kernel<RB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) set_for[dev] = (int)smem;
+    }
+    qkv_append_kernel<RB><<<p.nq + 2 * p.nk, kThreadsP, smem, st>>>(*tq, *tk, *tv, *th, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUtensorMap *tk,
+                              const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t st) {
+    ProjParams p = {};
+    p.h = static_cast<const __nv_bfloat16 *>(a.h);
+    p.q_out = static_cast<__nv_bfloat16 *>(a.q_out);
+    p.k_cache = static_cast<__nv_bfloat16 *>(a.k_cache);
+    p.v_cache = static_cast<__nv_bfloat16 *>(a.v_cache);
+    p.seqlens = a.seqlens;
+    p.seqlens_out = a.seqlens_out;
+    p.status = a.status;
+    p.B = a.B;
+    p.d = a.d;
+    p.H = a.H;
+    p.G = a.G;
+    p.d_h = a.d_h;
+    p.T_cap = a.T_cap;
+    p.nq = a.H * a.d_h / kNT;
+    p.nk = a.G * a.d_h / kNT;
+    p.timeout_ns = a.timeout_ns;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {  // 32 sequences per launch
+        p.b0 = b0;
+        const cudaError_t e =
+            (a.B - b0 > 16) ? run_proj<2>(p, tq, tk, tv, th, st) : run_proj<1>(p, tq, tk, tv, th, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace gqa

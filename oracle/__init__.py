@@ -75,6 +75,8 @@ def _load():
     lib.oracle_gqa_prefill_causal.restype = i32
     lib.oracle_meanpool.argtypes = [vp, i32, i32, i32, ctypes.c_size_t, vp]
     lib.oracle_meanpool.restype = i32
+    lib.oracle_project.argtypes = [vp, i32, vp, i32, vp, i32, i32, i32]
+    lib.oracle_project.restype = i32
     lib.oracle_round_bf16.argtypes = [vp, vp, ctypes.c_size_t]
     lib.oracle_round_bf16.restype = None
     lib.oracle_round_f32.argtypes = [vp, vp, ctypes.c_size_t]
@@ -229,3 +231,50 @@ def meanpool(W, G, out_dtype=None):
     """Mean-pool init: group means of W [H,d_h,d] rounded once to out_dtype."""
     mean = meanpool_mean(W, G)
     return round_to(mean, out_dtype or W.dtype)
+
+
+def project(h, W):
+    """fp64 h @ W: h [B, d], W [d, N] -> [B, N] (plain ascending-k sums)."""
+    lib = _load()
+    ht, hp, hdt = _as_host(h)
+    wt, wp, wdt = _as_host(W)
+    B, d = ht.shape
+    d2, N = wt.shape
+    if d != d2:
+        raise ValueError("h and W disagree on d")
+    out = torch.empty((B, N), dtype=torch.float64)
+    lib.oracle_project(hp, hdt, wp, wdt, out.data_ptr(), B, d, N)
+    return out
+
+
+def qkv_append(h, W_Q, W_K, W_V, k_cache, v_cache, seqlens):
+    """One decode token's projections and the cache append.
+
+    q = h @ W_Q -> [B, H, d_h]; k = h @ W_K, v = h @ W_V -> [B, G, d_h] (fp64),
+    written at position seqlens[b] of each sequence's cache, which then holds
+    one more token ("Grouped-Query Attention", section 1: the cache grows by
+    one key and one value vector per token, head and layer).  A sequence whose
+    cache is full (seqlens[b] >= T_cap) or whose length is negative gets no
+    append and keeps its length.
+
+    Returns (q, k, v, k_cache_after, v_cache_after, seqlens_after, appended)
+    where the caches after are float64 copies with the new rows in place.
+    """
+    Bq, d = h.shape
+    G, T_cap, d_h = k_cache.shape[1], k_cache.shape[2], k_cache.shape[3]
+    H = W_Q.shape[1] // d_h
+    q = project(h, W_Q).reshape(Bq, H, d_h)
+    k = project(h, W_K).reshape(Bq, G, d_h)
+    v = project(h, W_V).reshape(Bq, G, d_h)
+    kc = torch.as_tensor(k_cache).detach().cpu().double().clone()
+    vc = torch.as_tensor(v_cache).detach().cpu().double().clone()
+    sl = torch.as_tensor(seqlens).to(torch.int64).cpu().clone()
+    appended = torch.zeros(Bq, dtype=torch.bool)
+    for b in range(Bq):
+        t = int(sl[b])
+        if 0 <= t < T_cap:
+            kc[b, :, t, :] = k[b]
+            vc[b, :, t, :] = v[b]
+            sl[b] = t + 1
+            appended[b] = True
+    return q, k, v, kc, vc, sl.to(torch.int32), appended

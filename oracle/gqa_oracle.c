@@ -316,3 +316,22 @@ void oracle_round_bf16(const double *x, uint16_t *bits, size_t n) {
 void oracle_round_f32(const double *x, float *y, size_t n) {
     for (size_t i = 0; i < n; ++i) y[i] = (float)x[i];
 }
+
+/* ------------------------------------------------------------------ */
+/* projections of one token (decode step) and the KV-cache append      */
+/* ------------------------------------------------------------------ */
+
+/* out[b, n] = sum_k h[b, k] * W[k, n] in binary64 (ascending k).
+ * h [B, d]; W [d, N] row-major as in the sketch's h @ W ("Grouped-Query
+ * Attention", section 3: q = h @ W_Q, k = h @ W_K, v = h @ W_V). */
+int oracle_project(const void *h, int h_dt, const void *W, int w_dt, double *out, int B, int d,
+                   int N) {
+    for (int b = 0; b < B; ++b)
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < d; ++k)
+                acc += ld(h, h_dt, (size_t)b * d + k) * ld(W, w_dt, (size_t)k * N + n);
+            out[(size_t)b * N + n] = acc;
+        }
+    return 0;
+}

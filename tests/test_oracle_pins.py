@@ -381,3 +381,32 @@ def test_row_selection_rejects_out_of_range():
     p = gi.prefill_inputs(1, 4, 2, 1, 8, torch.float32, seed=18)
     with pytest.raises(IndexError):
         oracle.gqa_prefill_causal(p.q, p.k, p.v, p.scale, rows=[-1])
+
+
+# ----------------------------------------------------------------- projections
+
+def test_project_matches_torch_matmul_fp64():
+    x = gi.qkv_inputs(5, 64, 4, 2, 16, 4, seed=19)
+    got = oracle.project(x.h, x.W_Q)
+    assert (got - x.h.double() @ x.W_Q.double()).abs().max() < 1e-12
+
+
+def test_project_one_hot_rows_pick_weight_rows():
+    d, N = 32, 48
+    W = torch.randn(d, N, generator=torch.Generator().manual_seed(20)).to(torch.bfloat16)
+    h = torch.eye(d, dtype=torch.float64)[[3, 0, 31]]
+    assert torch.equal(oracle.project(h, W), W.double()[[3, 0, 31]])
+
+
+def test_qkv_append_grows_cache_by_2Gdh_scalars_per_token():
+    """KB s1/s2: one key and one value vector per KV head per token, i.e. the
+    closed form 2*G*d_h scalars; positions other than T_b stay as they were."""
+    x = gi.qkv_inputs(3, 64, 8, 2, 16, 5, seed=21, seqlens=[0, 4, 5])
+    q, k, v, kc, vc, sl, app = oracle.qkv_append(x.h, x.W_Q, x.W_K, x.W_V, x.k_cache, x.v_cache,
+                                                 x.seqlens)
+    assert app.tolist() == [True, True, False] and sl.tolist() == [1, 5, 5]
+    changed = ((kc != x.k_cache.double()).any(-1).sum() + (vc != x.v_cache.double()).any(-1).sum())
+    per_token_scalars = oracle.kv_cache_bytes(2, 16, 1, 1)
+    assert int(changed) * 16 == 2 * per_token_scalars            # two appends, G vectors each
+    assert q.shape == (3, 8, 16) and k.shape == (3, 2, 16)        # K/V GEMM is G/H of Q's
+    assert torch.equal(kc[0, :, 0], k[0]) and torch.equal(vc[1, :, 4], v[1])
