@@ -38,7 +38,9 @@ METRIC = "GQA decode achieved HBM GB/s (% of peak) & attn-tokens/s; prefill TFLO
 HEADLINE = "llama2_7b_decode"
 ROW_WORKLOADS = ["tiny_decode_fp32", "llama2_70b_ragged_decode"] + \
     ["long_ctx_decode_G%d" % g for g in (1, 2, 4, 8, 16, 32)] + ["causal_prefill", "meanpool_init",
-                                                                "qkv_append_llama2_7b"]
+                                                                "qkv_append_llama2_7b",
+                                                                "causal_prefill_window4096",
+                                                                "llama2_70b_ragged_decode_window4096"]
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, bytes, from ncu
 # captures of the current kernels (profiles/*.md); a workload missing here has
@@ -184,7 +186,11 @@ class Decode:
         self.ws = torch.empty(gqa.decode_workspace_bytes(x.B, x.H, x.G, x.d_h, x.T_cap, self.q.dtype),
                               dtype=torch.uint8, device=device)
         esz = self.q.element_size()
-        self.sum_T = int(x.seqlens.clamp(0, x.T_cap).sum())
+        self.window = w.get("window", 0)
+        T_att = x.seqlens.clamp(0, x.T_cap)
+        if self.window:
+            T_att = T_att.clamp(max=self.window)
+        self.sum_T = int(T_att.sum())                             # positions attended
         self.bytes = 2 * self.sum_T * x.G * x.d_h * esz           # K and V actually read
         self.flops = 4 * self.sum_T * x.H * x.d_h                 # q.k and p.v
         self.launches_per_step = 2
@@ -192,12 +198,12 @@ class Decode:
 
     def step(self, stream=None):
         self.gqa.decode(self.q, self.k, self.v, self.sl, self.x.scale, out=self.out,
-                        workspace=self.ws, stream=stream)
+                        workspace=self.ws, stream=stream, window=self.window)
 
     def config(self):
         x = self.x
         return {"workload": self.name, "B": x.B, "H": x.H, "G": x.G, "d_h": x.d_h, "T_cap": x.T_cap,
-                "sum_T": self.sum_T, "ragged": self.w["ragged"] is not None}
+                "sum_T": self.sum_T, "ragged": self.w["ragged"] is not None, "window": self.window}
 
     def metric(self, seconds_per_step, n_ranks):
         gbs = n_ranks * self.bytes / seconds_per_step / 1e9
@@ -242,12 +248,14 @@ class Decode:
                 kb, vb = x.k_cache[b:b + 1].cpu(), x.v_cache[b:b + 1].cpu()
                 t0 = time.perf_counter()
                 oracle.gqa_decode(x.q[b:b + 1].cpu(), kb, vb, x.seqlens[b:b + 1], x.scale,
-                                  rows=[r % x.H for r in rows])
+                                  rows=[r % x.H for r in rows], window=self.window)
             else:
                 t0 = time.perf_counter()
-                oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, rows=rows)
+                oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, rows=rows,
+                                  window=self.window)
             t_used += time.perf_counter() - t0
-            tokens += sum(int(x.seqlens[r // x.H].clamp(0, x.T_cap)) for r in rows)
+            tokens += sum(min(int(x.seqlens[r // x.H].clamp(0, x.T_cap)), self.window or x.T_cap)
+                          for r in rows)
             done += len(rows)
             n = min(2 * n, 512)
         # tokens here are (query head, key) pairs; convert to the step's KV bytes
@@ -267,18 +275,22 @@ class Prefill:
         self.q, self.k, self.v = x.q.to(device), x.k.to(device), x.v.to(device)
         self.out = torch.empty_like(self.q)
         S = x.S
-        self.flops = 4 * x.B * x.H * x.d_h * S * (S + 1) // 2      # causal QK^T + PV
+        self.window = w.get("window", 0)
+        Wn = self.window if self.window else S
+        pairs = sum(min(s + 1, Wn) for s in range(S))              # visible (query, key) pairs
+        self.flops = 4 * x.B * x.H * x.d_h * pairs                 # QK^T + PV on visible pairs
         self.bytes = (self.q.numel() * 2 + self.k.numel() * 2 * 2 + self.out.numel() * 2)
         self.launches_per_step = 1
         self.dtype = "bf16"
 
     def step(self, stream=None):
-        self.gqa.prefill_causal(self.q, self.k, self.v, self.x.scale, out=self.out, stream=stream)
+        self.gqa.prefill_causal(self.q, self.k, self.v, self.x.scale, out=self.out, stream=stream,
+                                window=self.window)
 
     def config(self):
         x = self.x
         return {"workload": self.name, "B": x.B, "S": x.S, "H": x.H, "G": x.G, "d_h": x.d_h,
-                "causal_flops": self.flops}
+                "causal_flops": self.flops, "window": self.window}
 
     def metric(self, sps, n_ranks):
         return {"value": n_ranks * self.flops / sps / 1e12, "unit": "TFLOP/s"}
@@ -300,9 +312,10 @@ class Prefill:
         while done < total and (done == 0 or t_used < budget_s):
             rows = torch.randint(0, total, (n,), generator=gen).tolist()
             t0 = time.perf_counter()
-            oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, rows=rows)
+            oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, rows=rows, window=self.window)
             t_used += time.perf_counter() - t0
-            flops += sum(4 * x.d_h * ((r // x.H) % x.S + 1) for r in rows)
+            Wn = self.window if self.window else x.S
+            flops += sum(4 * x.d_h * min((r // x.H) % x.S + 1, Wn) for r in rows)
             done += n
             n = min(2 * n, 1024)
         return {"seconds": t_used, "fraction_of_step": flops / self.flops,
@@ -517,21 +530,32 @@ def run_reference(args, world, rank):
 
 
 def make_host_only(name):
+    """A workload object with host inputs only (the reference arm needs no GPU)."""
     kind = gi.WORKLOADS[name]["kind"]
-    cls = {"decode": Decode, "prefill": Prefill, "meanpool": MeanPool}[kind]
+    cls = {"decode": Decode, "prefill": Prefill, "meanpool": MeanPool, "qkv": QkvAppend}[kind]
     obj = cls.__new__(cls)
     w = gi.WORKLOADS[name]
     obj.name, obj.w, obj.gqa = name, w, None
+    obj.window = w.get("window", 0)
     if kind == "decode":
         x = gi.decode_inputs(w["B"], w["H"], w["G"], w["d_h"], w["T"], w["dtype"], seed=0,
                              ragged=w["ragged"])
         obj.x = x
-        obj.sum_T = int(x.seqlens.clamp(0, x.T_cap).sum())
+        T_att = x.seqlens.clamp(0, x.T_cap)
+        if obj.window:
+            T_att = T_att.clamp(max=obj.window)
+        obj.sum_T = int(T_att.sum())
         obj.bytes = 2 * obj.sum_T * x.G * x.d_h * x.q.element_size()
     elif kind == "prefill":
         x = gi.prefill_inputs(w["B"], w["S"], w["H"], w["G"], w["d_h"], w["dtype"], seed=0)
         obj.x = x
-        obj.flops = 4 * x.B * x.H * x.d_h * x.S * (x.S + 1) // 2
+        Wn = obj.window if obj.window else x.S
+        obj.flops = 4 * x.B * x.H * x.d_h * sum(min(s + 1, Wn) for s in range(x.S))
+    elif kind == "qkv":
+        x = gi.qkv_inputs(w["B"], w["d"], w["H"], w["G"], w["d_h"], w["T"], w["dtype"], seed=0)
+        obj.x = x
+        obj.bytes = (x.d * (x.H + 2 * x.G) * x.d_h + x.B * x.d + x.B * x.H * x.d_h
+                     + 2 * x.B * x.G * x.d_h) * x.h.element_size()
     else:
         wk, wv = gi.meanpool_inputs(w["H"], w["d_h"], w["d"], w["dtype"], seed=0, std=w["std"])
         obj.wk_h, obj.wv_h = wk, wv

@@ -29,6 +29,12 @@ WORKLOADS = {
                            dtype=torch.bfloat16),
     "meanpool_init": dict(kind="meanpool", H=64, G=8, d_h=128, d=8192,
                           dtype=torch.bfloat16, std=0.02),
+    # sliding-window variants (4096-key window)
+    "causal_prefill_window4096": dict(kind="prefill", B=2, S=8192, H=64, G=8, d_h=128,
+                                      dtype=torch.bfloat16, window=4096),
+    "llama2_70b_ragged_decode_window4096": dict(kind="decode", B=32, H=64, G=8, d_h=128, T=8192,
+                                                dtype=torch.bfloat16, ragged=(1024, 8192),
+                                                window=4096),
     # one decode token's projections + cache append, Llama-2-7B shape (d = 4096)
     "qkv_append_llama2_7b": dict(kind="qkv", B=16, d=4096, H=32, G=8, d_h=128, T=4096,
                                  dtype=torch.bfloat16),

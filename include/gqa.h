@@ -110,6 +110,19 @@ GQA_API int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                size_t workspace_bytes, gqa_stream_t stream);
 
 /*
+ * gqa_decode_window -- gqa_decode with a sliding window: each sequence
+ * attends over its last min(T_b, window) cached positions only,
+ * [T_b - window, T_b), instead of all T_b ("Grouped-Query Attention",
+ * llm-arch-kb, section 4: Mistral 7B pairs GQA with sliding-window
+ * attention).  window = 0 is gqa_decode.  Same arguments, workspace and
+ * limits as gqa_decode; window < 0 is GQA_ERR_INVALID.
+ */
+GQA_API int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *seqlens, float scale, void *out, int B, int H,
+                              int G, int d_h, int T_cap, int window, gqa_dtype dt,
+                              void *workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/*
  * gqa_decode_noalloc -- gqa_decode for callers that cannot allocate device
  * memory.  (The pages have no counterpart: this is a deployment convenience.)
  *
@@ -157,6 +170,16 @@ GQA_API int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v
 GQA_API int gqa_prefill_causal(const void *q, const void *k, const void *v, void *out,
                        int B, int S, int H, int G, int d_h, float scale,
                        gqa_dtype dt, gqa_stream_t stream);
+
+/*
+ * gqa_prefill_causal_window -- causal prefill with a sliding window of
+ * `window` keys: query s sees keys s - window < t <= s (itself and the
+ * window - 1 before it); KV tiles wholly outside every row's window are not
+ * read.  window = 0 is gqa_prefill_causal.  Same arguments and limits.
+ */
+GQA_API int gqa_prefill_causal_window(const void *q, const void *k, const void *v, void *out,
+                                      int B, int S, int H, int G, int d_h, float scale,
+                                      int window, gqa_dtype dt, gqa_stream_t stream);
 
 /*
  * gqa_meanpool_kv -- averaging initialisation of GQA key/value projections

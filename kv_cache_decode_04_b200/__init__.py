@@ -34,8 +34,9 @@ _ERRORS = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGN", -4: "CUDA", -5: "WORKS
 
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_kv_cache_bytes", "gqa_decode_workspace_bytes", "gqa_decode",
-           "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_qkv_append",
-           "gqa_get_status", "gqa_last_error_string", "gqa_version")
+           "gqa_decode_window", "gqa_decode_noalloc", "gqa_prefill_causal",
+           "gqa_prefill_causal_window", "gqa_meanpool_kv", "gqa_qkv_append", "gqa_get_status",
+           "gqa_last_error_string", "gqa_version")
 
 
 class GQAError(RuntimeError):
@@ -56,6 +57,12 @@ def _load():
     L.gqa_decode_workspace_bytes.restype = sz
     L.gqa_decode.argtypes = [vp, vp, vp, vp, f32, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]
     L.gqa_decode.restype = i32
+    L.gqa_decode_window.argtypes = [vp, vp, vp, vp, f32, vp, i32, i32, i32, i32, i32, i32, i32, vp,
+                                    sz, vp]
+    L.gqa_decode_window.restype = i32
+    L.gqa_prefill_causal_window.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, i32,
+                                            vp]
+    L.gqa_prefill_causal_window.restype = i32
     L.gqa_decode_noalloc.argtypes = [vp, vp, vp, vp, f32, vp, i32, i32, i32, i32, i32, i32, vp]
     L.gqa_decode_noalloc.restype = i32
     L.gqa_prefill_causal.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, vp]
@@ -115,11 +122,13 @@ def decode_workspace_bytes(B, H, G, d_h, T_cap, dtype=torch.bfloat16) -> int:
     return n
 
 
-def decode(q, k_cache, v_cache, seqlens, scale=None, out=None, workspace=None, stream=None):
+def decode(q, k_cache, v_cache, seqlens, scale=None, out=None, workspace=None, stream=None,
+           window=0):
     """GQA decode: out[b,i] = softmax(scale q[b,i].K[b,g]^T over t < seqlens[b]) V[b,g].
 
     q [B,H,d_h]; k_cache, v_cache [B,G,T_cap,d_h]; seqlens [B] int32 (device);
-    scale defaults to 1/sqrt(d_h).  Returns ``out`` [B,H,d_h].
+    scale defaults to 1/sqrt(d_h).  window > 0 attends over the last
+    ``window`` cached positions only.  Returns ``out`` [B,H,d_h].
     """
     B, H, d_h = q.shape
     Bk, G, T_cap, dk = k_cache.shape
@@ -137,10 +146,10 @@ def decode(q, k_cache, v_cache, seqlens, scale=None, out=None, workspace=None, s
     if workspace is None:  # (a given workspace's size is checked by the library)
         need = decode_workspace_bytes(B, H, G, d_h, T_cap, q.dtype)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    rc = lib.gqa_decode(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-                        _dev(seqlens, "seqlens"), float(scale), _dev(out, "out"), B, H, G, d_h,
-                        T_cap, code, _dev(workspace, "workspace"), workspace.numel(),
-                        _stream(stream))
+    rc = lib.gqa_decode_window(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                               _dev(seqlens, "seqlens"), float(scale), _dev(out, "out"), B, H, G,
+                               d_h, T_cap, int(window), code, _dev(workspace, "workspace"),
+                               workspace.numel(), _stream(stream))
     _check(rc)
     return out
 
@@ -171,8 +180,11 @@ def decode_noalloc(q, k_cache, v_cache, seqlens, scale=None, out=None, stream=No
     return out
 
 
-def prefill_causal(q, k, v, scale=None, out=None, stream=None):
-    """Causal GQA prefill: q [B,S,H,d_h], k/v [B,S,G,d_h] bf16 -> out [B,S,H,d_h]."""
+def prefill_causal(q, k, v, scale=None, out=None, stream=None, window=0):
+    """Causal GQA prefill: q [B,S,H,d_h], k/v [B,S,G,d_h] bf16 -> out [B,S,H,d_h].
+
+    window > 0: query s sees keys s-window < t <= s only.
+    """
     B, S, H, d_h = q.shape
     G = k.shape[2]
     if tuple(k.shape) != (B, S, G, d_h) or tuple(v.shape) != tuple(k.shape):
@@ -182,8 +194,9 @@ def prefill_causal(q, k, v, scale=None, out=None, stream=None):
         scale = 1.0 / math.sqrt(d_h)
     if out is None:
         out = torch.empty_like(q)
-    rc = lib.gqa_prefill_causal(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
-                                B, S, H, G, d_h, float(scale), code, _stream(stream))
+    rc = lib.gqa_prefill_causal_window(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
+                                       B, S, H, G, d_h, float(scale), int(window), code,
+                                       _stream(stream))
     _check(rc)
     return out
 

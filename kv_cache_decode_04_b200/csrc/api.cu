@@ -154,11 +154,12 @@ size_t gqa_decode_workspace_bytes(int B, int H, int G, int d_h, int T_cap, gqa_d
     return gqa::decode_layout(B, H, G, d_h, T_cap, dt, d->num_sms, forced_splits()).total;
 }
 
-int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
-               float scale, void *out, int B, int H, int G, int d_h, int T_cap, gqa_dtype dt,
-               void *workspace, size_t workspace_bytes, gqa_stream_t stream) {
+static int decode_impl(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                       float scale, void *out, int B, int H, int G, int d_h, int T_cap, int window,
+                       gqa_dtype dt, void *workspace, size_t workspace_bytes, gqa_stream_t stream) {
     t_err[0] = 0;
     int rc = check_dims(B, H, G, d_h);
+    if (window < 0) return fail(GQA_ERR_INVALID, "window must be >= 0 (0: no window)");
     if (rc) return rc;
     if (T_cap <= 0) return fail(GQA_ERR_INVALID, "T_cap must be positive");
     if (!q || !k_cache || !v_cache || !seqlens || !out) return fail(GQA_ERR_INVALID, "null tensor pointer");
@@ -215,15 +216,31 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
     a.timeout_ns = wait_timeout_ns();
     a.num_sms = d->num_sms;
     a.force_ctas = forced_splits();
+    a.window = window;
     cudaError_t e = gqa::launch_decode(a, &tmk, &tmv, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "decode launch");
     return GQA_OK;
 }
 
-int gqa_prefill_causal(const void *q, const void *k, const void *v, void *out, int B, int S, int H,
-                       int G, int d_h, float scale, gqa_dtype dt, gqa_stream_t stream) {
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+               float scale, void *out, int B, int H, int G, int d_h, int T_cap, gqa_dtype dt,
+               void *workspace, size_t workspace_bytes, gqa_stream_t stream) {
+    return decode_impl(q, k_cache, v_cache, seqlens, scale, out, B, H, G, d_h, T_cap, 0, dt, workspace,
+                       workspace_bytes, stream);
+}
+
+int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                      float scale, void *out, int B, int H, int G, int d_h, int T_cap, int window,
+                      gqa_dtype dt, void *workspace, size_t workspace_bytes, gqa_stream_t stream) {
+    return decode_impl(q, k_cache, v_cache, seqlens, scale, out, B, H, G, d_h, T_cap, window, dt, workspace,
+                       workspace_bytes, stream);
+}
+
+static int prefill_impl(const void *q, const void *k, const void *v, void *out, int B, int S, int H, int G,
+                        int d_h, float scale, int window, gqa_dtype dt, gqa_stream_t stream) {
     t_err[0] = 0;
     int rc = check_dims(B, H, G, d_h);
+    if (window < 0) return fail(GQA_ERR_INVALID, "window must be >= 0 (0: no window)");
     if (rc) return rc;
     if (S <= 0) return fail(GQA_ERR_INVALID, "S must be positive");
     if (!q || !k || !v || !out) return fail(GQA_ERR_INVALID, "null tensor pointer");
@@ -273,9 +290,20 @@ int gqa_prefill_causal(const void *q, const void *k, const void *v, void *out, i
     a.status = d->status;
     a.timeout_ns = wait_timeout_ns();
     a.num_sms = d->num_sms;
+    a.window = window;
     cudaError_t e = gqa::launch_prefill(a, &tmq, &tmk, &tmv, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "prefill launch");
     return GQA_OK;
+}
+
+int gqa_prefill_causal(const void *q, const void *k, const void *v, void *out, int B, int S, int H, int G,
+                       int d_h, float scale, gqa_dtype dt, gqa_stream_t stream) {
+    return prefill_impl(q, k, v, out, B, S, H, G, d_h, scale, 0, dt, stream);
+}
+
+int gqa_prefill_causal_window(const void *q, const void *k, const void *v, void *out, int B, int S, int H,
+                              int G, int d_h, float scale, int window, gqa_dtype dt, gqa_stream_t stream) {
+    return prefill_impl(q, k, v, out, B, S, H, G, d_h, scale, window, dt, stream);
 }
 
 int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *WV_out, int H, int G, int d_h,

@@ -58,10 +58,18 @@ struct DecodeParams {
     float scale_log2;
     int B, H, G, r, T_cap;
     unsigned long long timeout_ns;
+    int window;  // > 0: attend over the last `window` cached positions only
 };
 
 __device__ __forceinline__ int clamp_len(int T, int T_cap) {
     return T < 0 ? 0 : (T > T_cap ? T_cap : T);
+}
+
+// Cached positions a sequence attends over: all T_b of them, or with a sliding
+// window of W > 0 only the last min(T_b, W), i.e. [T_b - len, T_b).
+__device__ __forceinline__ int attended_len(int T, const DecodeParams &p) {
+    const int t = clamp_len(T, p.T_cap);
+    return (p.window > 0 && t > p.window) ? p.window : t;
 }
 
 // cu[b] = G * sum_{b' < b} ceil(T_b' / TILE), T clamped to [0, T_cap];
@@ -77,7 +85,7 @@ __device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, b
     for (int b = b0; b < b1; ++b) {
         const int T = p.seqlens[b];
         bad |= (T < 0 || T > p.T_cap);
-        local += (clamp_len(T, p.T_cap) + TILE - 1) / TILE;
+        local += (attended_len(T, p) + TILE - 1) / TILE;
     }
     if (bad && report) set_status(p.status, STATUS_SEQLEN);
     // exclusive block scan of `local`: warp scans, then a scan of the warp totals
@@ -104,7 +112,7 @@ __device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, b
     int run = incl - local + (wid > 0 ? scratch[wid - 1] : 0);
     for (int b = b0; b < b1; ++b) {
         cu[b] = run * p.G;
-        run += (clamp_len(p.seqlens[b], p.T_cap) + TILE - 1) / TILE;
+        run += (attended_len(p.seqlens[b], p) + TILE - 1) / TILE;
     }
     __syncthreads();
     return cu[p.B];
@@ -221,7 +229,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 uint8_t *kdst = stages + s * STAGE_BYTES;
                 uint8_t *vdst = kdst + KV_BYTES;
                 mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-                const int row = (c.b * p.G + c.g) * p.T_cap + c.j * kTile;
+                const int Tb = clamp_len(p.seqlens[c.b], p.T_cap);
+                const int start = Tb - attended_len(Tb, p);
+                const int row = (c.b * p.G + c.g) * p.T_cap + start + c.j * kTile;
 #pragma unroll
                 for (int h = 0; h < HALVES; ++h) {
                     tma_load_2d(kdst + h * kHalfBytes, &tmk, &full[s], h * 64, row, pol);
@@ -248,9 +258,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     cursor_seek(cu, p.B, p.G, u_begin, c);
     for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
         const int b = c.b, bg = c.b * p.G + c.g;
-        const int t0 = c.j * kTile;
-        const int seq_len = clamp_len(p.seqlens[b], p.T_cap);
-        const int n_valid = min(kTile, seq_len - t0);
+        const int seq_len = attended_len(p.seqlens[b], p);  // tiles start at T_b - seq_len
+        const int n_valid = min(kTile, seq_len - c.j * kTile);
         if (bg != cur_bg) {  // first tile of a piece: this group's queries
             cur_bg = bg;
             const int hl_a = mt * 16 + g8, hl_b = hl_a + 8;
@@ -495,8 +504,9 @@ __global__ void __launch_bounds__(kThreadsF32)
     cursor_seek(cu, p.B, p.G, u_begin, c);
     for (int u = u_begin; u < u_end; ++u) {
         const int b = c.b, bg = c.b * p.G + c.g;
-        const int t0 = c.j * kTileF32;
-        const int n_valid = min(kTileF32, clamp_len(p.seqlens[b], p.T_cap) - t0);
+        const int seq_len = attended_len(p.seqlens[b], p);
+        const int t0 = clamp_len(p.seqlens[b], p.T_cap) - seq_len + c.j * kTileF32;
+        const int n_valid = min(kTileF32, seq_len - c.j * kTileF32);
         if (bg != cur_bg) {
             cur_bg = bg;
             const float *qb = qg + ((size_t)b * p.H + (size_t)c.g * p.r) * D;
@@ -755,6 +765,7 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUt
     p.r = a.H / a.G;
     p.T_cap = a.T_cap;
     p.timeout_ns = a.timeout_ns;
+    p.window = a.window;
     cudaError_t e;
     if (a.dtype == GQA_BF16) {
         const int nmt = bf16_nmt(p.r);

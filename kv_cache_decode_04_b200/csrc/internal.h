@@ -26,6 +26,7 @@ struct DecodeArgs {
     uint64_t timeout_ns;
     int num_sms;
     int force_ctas;  // >0: use this many split CTAs (tests of the split logic)
+    int window;      // >0: sliding window of the last `window` cached positions
 };
 
 // Workspace layout, all offsets 256-byte aligned.
@@ -50,6 +51,7 @@ struct PrefillArgs {
     unsigned *status;
     uint64_t timeout_ns;
     int num_sms;
+    int window;  // >0: query s sees keys s-window < t <= s
 };
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const CUtensorMap *tmk,
                            const CUtensorMap *tmv, cudaStream_t stream);

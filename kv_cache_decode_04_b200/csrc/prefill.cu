@@ -25,6 +25,8 @@
 // the same because numerator and denominator use the same stale maximum.
 // Only KV tiles j <= query tile are visited; the diagonal tile is masked
 // (key > query -> -inf).
+#include <climits>
+
 #include "common.cuh"
 #include "exp2_fma.cuh"
 #include "gqa.h"
@@ -62,6 +64,7 @@ struct PrefillParams {
     float scale_log2;
     int B, S, H, G, r, n_qt;
     unsigned long long timeout_ns;
+    int window;  // > 0: query s sees keys s - window < t <= s
 };
 
 __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, uint64_t *bar, int x, int y,
@@ -131,7 +134,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = (rem / pairs) % p.G;
     const int h0 = g * p.r + 2 * (rem % pairs);
     const int s0 = qt * kBM;
-    const int n_kv = qt + 1;
+    // KV tiles j_lo..qt: with a sliding window of W keys the tiles wholly below the
+    // first row's window (keys < s0 - W + 1) are skipped.
+    const int j_lo = p.window > 0 ? max(0, s0 - p.window + 1) / kBN : 0;
+    const int n_kv = qt - j_lo + 1;
+    // Rows that see few keys carry P as two bf16 terms (see the softmax below).
+    const bool split_p = qt == 0 || (p.window > 0 && p.window <= 256);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -169,9 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int half = 0; half < 2; ++half)
                     tma_load_4d(sm + kOffQ + hh * kTile + half * kHalf, &tmq, bar_q, half * 64, h0 + hh, s0,
                                 b, pol_q);
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
+            for (int jj = 0; jj < n_kv; ++jj) {
+                const int j = j_lo + jj;
+                const int st = jj & 1;
+                const uint32_t ph = (jj >> 1) & 1;
                 if (*vabort || !mbar_wait(&k_empty[st], ph ^ 1, p.timeout_ns)) {
                     set_status(p.status, STATUS_TIMEOUT);
                     *vabort = 1;
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // O_h += P_h V: 8 K-steps of 16 keys; V is MN-major (d_h contiguous).  On
             // the first query tile a second pass adds P_lo (TMEM columns 64..127).
             auto issue_pv = [&](int hh, int vs, bool acc) {
-                const int passes = qt == 0 ? 2 : 1;
+                const int passes = split_p ? 2 : 1;
 #pragma unroll 1
                 for (int ps = 0; ps < passes; ++ps)
 #pragma unroll
@@ -243,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::commit(&s_full[1]);
                 tc::commit(&k_empty[0]);
                 issued = true;
-                for (int j = 0; j < n_kv && ok; ++j) {
+                for (int j = 0; j < n_kv && ok; ++j) {  // j counts visited tiles
                     const int st = j & 1;
                     const uint32_t ph = (j >> 1) & 1;
                     const int st2 = (j + 1) & 1;
@@ -286,10 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tO = tmem + lane_off + 256 + hh * 128;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        const bool split_p = (qt == 0);
-        for (int j = 0; j < n_kv; ++j) {
+        // first key this row may see under a sliding window (none below it)
+        const int key_lo = p.window > 0 ? s0 + t - p.window + 1 : INT_MIN;
+        for (int jj = 0; jj < n_kv; ++jj) {
+            const int j = j_lo + jj;  // KV tile index
             const bool aborted = __any_sync(0xffffffffu, *vabort != 0);  // warp-uniform
-            if (aborted || !warp_wait(&s_full[hh], j & 1, p.timeout_ns)) {
+            if (aborted || !warp_wait(&s_full[hh], jj & 1, p.timeout_ns)) {
                 if (lane == 0) set_status(p.status, STATUS_TIMEOUT);
                 *vabort = 1;
                 ok = false;
@@ -300,13 +311,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, sr[c]);
             tc::wait_ld();
-            const bool diag = (j == n_kv - 1);
-            if (diag) {  // keys after the query row are masked
+            const bool diag = (j == qt);
+            // a tile holding keys below some row's window start
+            const bool lo_tile = p.window > 0 && j * kBN < s0 + kBM - p.window;
+            if (diag || lo_tile) {  // keys after the query row, or before its window, are masked
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (c * 32 + e > t) sr[c][e] = __float_as_uint(-INFINITY);
+                    for (int e = 0; e < 32; ++e) {
+                        const int key = j * kBN + c * 32 + e;
+                        if ((diag && key > s0 + t) || key < key_lo) sr[c][e] = __float_as_uint(-INFINITY);
+                    }
             }
             // Row maximum of the raw scores (the scale is positive), with eight
             // independent partial maxima instead of one 128-long chain.
@@ -321,8 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
             float alpha = 1.f;
             bool rescale = false;
-            if (j == 0) {
-                m = mx;  // key 0 is always visible, so mx is finite
+            if (jj == 0) {
+                m = mx;  // -inf when a sliding window hides this tile from the row
             } else {
                 const float mn = fmaxf(m, mx);
                 const bool need = mn > m + 8.f;
@@ -339,10 +354,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Rows of the first query tile see at most 128 keys, too few for the bf16
             // rounding of P to average out; there P is carried as P_hi + P_lo (two bf16
             // terms, about 16 significant bits), P_lo in columns 64..127.
+            // a row that has seen no key yet (m = -inf) has only -inf scores: p = 0
+            const float mu = m == -INFINITY ? 0.f : m;
             const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2);
-            const uint64_t nm2 = f32x2_pack(-m, -m);
+            const uint64_t nm2 = f32x2_pack(-mu, -mu);
             uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
-            if (!split_p && !diag) {
+            if (!split_p && !diag && !lo_tile) {
                 // Off-diagonal tiles: one exponential in four on the FMA pipe
                 // (exp2_fma), the rest on the special-function unit.
 #pragma unroll
@@ -384,8 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int e1 = 0; e1 < 4; ++e1) {
                             const int e = e4 * 4 + e1;
-                            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e]), p.scale_log2, -m));
-                            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e + 1]), p.scale_log2, -m));
+                            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e]), p.scale_log2, -mu));
+                            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e + 1]), p.scale_log2, -mu));
                             rs2[e1] = f32x2_add(rs2[e1], f32x2_pack(p0, p1));
                             ph[e1] = pack_bf16x2(p0, p1);
                             const float2 h = unpack_bf16x2(ph[e1]);
@@ -468,6 +485,7 @@ cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const C
     p.G = a.G;
     p.r = a.H / a.G;
     p.n_qt = (a.S + kBM - 1) / kBM;
+    p.window = a.window;
     p.timeout_ns = a.timeout_ns;
     const long long grid = (long long)p.n_qt * a.B * a.G * (p.r / 2);
     if (grid <= 0 || grid >= (1ll << 31)) return cudaErrorInvalidConfiguration;

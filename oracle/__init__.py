@@ -65,13 +65,13 @@ def _load():
     lib.oracle_kv_cache_bytes.restype = ctypes.c_uint64
     lib.oracle_default_threads.restype = i32
     lib.oracle_gqa_decode.argtypes = [vp, i32, vp, vp, i32, vp, dbl, vp,
-                                      i32, i32, i32, i32, i32, vp, i64, i32]
+                                      i32, i32, i32, i32, i32, vp, i64, i32, i32]
     lib.oracle_gqa_decode.restype = i32
     lib.oracle_mha_decode.argtypes = [vp, i32, vp, vp, i32, vp, dbl, vp,
                                       i32, i32, i32, i32, i32]
     lib.oracle_mha_decode.restype = i32
     lib.oracle_gqa_prefill_causal.argtypes = [vp, vp, vp, i32, dbl, vp, i32, i32,
-                                              i32, i32, i32, vp, i64, i32]
+                                              i32, i32, i32, vp, i64, i32, i32]
     lib.oracle_gqa_prefill_causal.restype = i32
     lib.oracle_meanpool.argtypes = [vp, i32, i32, i32, ctypes.c_size_t, vp]
     lib.oracle_meanpool.restype = i32
@@ -133,10 +133,11 @@ def kv_cache_bytes(G: int, d_h: int, L: int, elem_bytes: int) -> int:
     return int(_load().oracle_kv_cache_bytes(int(G), int(d_h), int(L), int(elem_bytes)))
 
 
-def gqa_decode(q, k_cache, v_cache, seqlens, scale, rows=None, nthreads=0):
+def gqa_decode(q, k_cache, v_cache, seqlens, scale, rows=None, nthreads=0, window=0):
     """fp64 GQA decode.
 
     q [B,H,d_h]; k_cache, v_cache [B,G,T_cap,d_h]; seqlens [B] ints.
+    window > 0: attend over the last `window` cached positions only.
     Returns float64 [B,H,d_h], or [len(rows), d_h] for rows = flat (b*H + i).
     """
     lib = _load()
@@ -151,7 +152,7 @@ def gqa_decode(q, k_cache, v_cache, seqlens, scale, rows=None, nthreads=0):
     rt, rp, nr = _rows(rows, B * H)
     out = torch.empty((nr, d_h) if rt is not None else (B, H, d_h), dtype=torch.float64)
     rc = lib.oracle_gqa_decode(qp, qdt, kp, vp_, kdt, sp, float(scale), out.data_ptr(),
-                               B, H, G, d_h, T_cap, rp, nr, int(nthreads))
+                               B, H, G, d_h, T_cap, rp, nr, int(nthreads), int(window))
     if rc != 0:
         raise ValueError("oracle_gqa_decode failed (rc=%d)" % rc)
     return out
@@ -176,11 +177,12 @@ def mha_decode(q, k_cache, v_cache, seqlens, scale, nthreads=0):
     return out
 
 
-def gqa_prefill_causal(q, k, v, scale, rows=None, nthreads=0):
+def gqa_prefill_causal(q, k, v, scale, rows=None, nthreads=0, window=0):
     """fp64 causal GQA prefill.
 
-    q [B,S,H,d_h]; k, v [B,S,G,d_h] (same dtype).  Returns float64
-    [B,S,H,d_h], or [len(rows), d_h] for rows = flat ((b*S + s)*H + i).
+    q [B,S,H,d_h]; k, v [B,S,G,d_h] (same dtype).  window > 0: query s sees
+    keys s-window < t <= s.  Returns float64 [B,S,H,d_h], or [len(rows), d_h]
+    for rows = flat ((b*S + s)*H + i).
     """
     lib = _load()
     qt, qp, qdt = _as_host(q)
@@ -193,7 +195,7 @@ def gqa_prefill_causal(q, k, v, scale, rows=None, nthreads=0):
     rt, rp, nr = _rows(rows, B * S * H)
     out = torch.empty((nr, d_h) if rt is not None else (B, S, H, d_h), dtype=torch.float64)
     rc = lib.oracle_gqa_prefill_causal(qp, kp, vp_, qdt, float(scale), out.data_ptr(),
-                                       B, S, H, G, d_h, rp, nr, int(nthreads))
+                                       B, S, H, G, d_h, rp, nr, int(nthreads), int(window))
     if rc != 0:
         raise ValueError("oracle_gqa_prefill_causal failed (rc=%d)" % rc)
     return out

@@ -24,6 +24,9 @@
  *   - decode attends over exactly seqlens[b] cached positions; an empty
  *     cache (seqlens[b] == 0) yields a zero output row;
  *   - the causal mask keeps key t for query s when t <= s (diagonal kept);
+ *   - a sliding window of W keys (section 4 names sliding-window attention
+ *     alongside GQA for Mistral 7B) keeps, for prefill query s, the keys
+ *     s - W < t <= s, and for decode the last W cached positions;
  *   - softmax is evaluated in two plain passes (maximum, then exp/sum);
  *     there is no running rescale and no split of the key axis.
  *
@@ -179,6 +182,7 @@ typedef struct {
     int kv_heads;          /* G for GQA, H for per-head MHA */
     int per_head_kv;       /* 1: head i reads KV head i (MHA)  */
     const int64_t *rows;   /* optional list of (b*H + i) rows */
+    int window;            /* > 0: only the last `window` cached positions */
 } dec_ctx;
 
 static void decode_unit(void *vc, long u, double *s) {
@@ -188,9 +192,12 @@ static void decode_unit(void *vc, long u, double *s) {
     int kvh = c->per_head_kv ? i : oracle_group_of_head(i, c->H, c->G);
     long n = c->seqlens[b];
     if (n > c->T_cap) n = c->T_cap;
+    if (n < 0) n = 0;
+    long first = 0; /* first cached position attended */
+    if (c->window > 0 && n > c->window) first = n - c->window;
     size_t q_off = ((size_t)b * c->H + i) * c->d_h;
-    size_t kv_off = (((size_t)b * c->kv_heads + kvh) * c->T_cap) * c->d_h;
-    attend_row(c->q, q_off, c->K, kv_off, c->V, kv_off, (size_t)c->d_h, n,
+    size_t kv_off = ((((size_t)b * c->kv_heads + kvh) * c->T_cap) + (size_t)first) * c->d_h;
+    attend_row(c->q, q_off, c->K, kv_off, c->V, kv_off, (size_t)c->d_h, n - first,
                c->d_h, c->scale, c->out + (size_t)u * c->d_h, s);
 }
 
@@ -199,10 +206,10 @@ static void decode_unit(void *vc, long u, double *s) {
 int oracle_gqa_decode(const void *q, int q_dt, const void *K, const void *V,
                       int kv_dt, const int32_t *seqlens, double scale,
                       double *out, int B, int H, int G, int d_h, int T_cap,
-                      const int64_t *rows, long n_rows, int nthreads) {
+                      const int64_t *rows, long n_rows, int nthreads, int window) {
     if (G <= 0 || H % G != 0) return -1;
     dec_ctx c = {{q, q_dt}, {K, kv_dt}, {V, kv_dt}, seqlens, scale, out,
-                 B, H, G, d_h, T_cap, G, 0, rows};
+                 B, H, G, d_h, T_cap, G, 0, rows, window};
     long n = rows ? n_rows : (long)B * H;
     return run_pool(decode_unit, &c, n, (size_t)T_cap, nthreads);
 }
@@ -213,7 +220,7 @@ int oracle_mha_decode(const void *q, int q_dt, const void *K, const void *V,
                       double *out, int B, int H, int d_h, int T_cap,
                       int nthreads) {
     dec_ctx c = {{q, q_dt}, {K, kv_dt}, {V, kv_dt}, seqlens, scale, out,
-                 B, H, H, d_h, T_cap, H, 1, NULL};
+                 B, H, H, d_h, T_cap, H, 1, NULL, 0};
     return run_pool(decode_unit, &c, (long)B * H, (size_t)T_cap, nthreads);
 }
 
@@ -227,6 +234,7 @@ typedef struct {
     double *out;
     int B, S, H, G, d_h;
     const int64_t *rows; /* optional list of ((b*S + s)*H + i) */
+    int window;          /* > 0: keys s - window < t <= s */
 } pre_ctx;
 
 static void prefill_unit(void *vc, long u, double *sc) {
@@ -237,10 +245,11 @@ static void prefill_unit(void *vc, long u, double *sc) {
     int s = (int)(bs % c->S), b = (int)(bs / c->S);
     int g = oracle_group_of_head(i, c->H, c->G);
     size_t q_off = (((size_t)b * c->S + s) * c->H + i) * c->d_h;
-    size_t kv_off = (((size_t)b * c->S + 0) * c->G + g) * c->d_h;
+    long first = 0; /* causal mask: query s sees keys first..s */
+    if (c->window > 0 && (long)s + 1 > c->window) first = (long)s + 1 - c->window;
+    size_t kv_off = (((size_t)b * c->S + (size_t)first) * c->G + g) * c->d_h;
     size_t stride = (size_t)c->G * c->d_h; /* token-major k/v */
-    /* causal mask: query s sees keys 0..s */
-    attend_row(c->q, q_off, c->k, kv_off, c->v, kv_off, stride, (long)s + 1,
+    attend_row(c->q, q_off, c->k, kv_off, c->v, kv_off, stride, (long)s + 1 - first,
                c->d_h, c->scale, c->out + (size_t)u * c->d_h, sc);
 }
 
@@ -249,9 +258,9 @@ static void prefill_unit(void *vc, long u, double *sc) {
 int oracle_gqa_prefill_causal(const void *q, const void *k, const void *v,
                               int dt, double scale, double *out, int B, int S,
                               int H, int G, int d_h, const int64_t *rows,
-                              long n_rows, int nthreads) {
+                              long n_rows, int nthreads, int window) {
     if (G <= 0 || H % G != 0) return -1;
-    pre_ctx c = {{q, dt}, {k, dt}, {v, dt}, scale, out, B, S, H, G, d_h, rows};
+    pre_ctx c = {{q, dt}, {k, dt}, {v, dt}, scale, out, B, S, H, G, d_h, rows, window};
     long n = rows ? n_rows : (long)B * S * H;
     return run_pool(prefill_unit, &c, n, (size_t)S, nthreads);
 }

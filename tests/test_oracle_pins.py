@@ -410,3 +410,48 @@ def test_qkv_append_grows_cache_by_2Gdh_scalars_per_token():
     assert int(changed) * 16 == 2 * per_token_scalars            # two appends, G vectors each
     assert q.shape == (3, 8, 16) and k.shape == (3, 2, 16)        # K/V GEMM is G/H of Q's
     assert torch.equal(kc[0, :, 0], k[0]) and torch.equal(vc[1, :, 4], v[1])
+
+
+# ----------------------------------------------------------------- sliding window
+
+def _band_sdpa_prefill(x, W):
+    """SDPA in float64 with an explicit band mask: key t visible to s iff s-W < t <= s."""
+    S = x.S
+    s = torch.arange(S)[:, None]
+    t = torch.arange(S)[None, :]
+    mask = (t <= s) & (t > s - W)
+    q = x.q.double().permute(0, 2, 1, 3)
+    k = x.k.double().permute(0, 2, 1, 3)
+    v = x.v.double().permute(0, 2, 1, 3)
+    o = F.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=x.scale, enable_gqa=True)
+    return o.permute(0, 2, 1, 3)
+
+
+@pytest.mark.parametrize("W", [1, 5, 16, 40])
+def test_prefill_window_matches_band_masked_sdpa(W):
+    x = gi.prefill_inputs(2, 40, 8, 2, 16, torch.bfloat16, seed=22 + W)
+    got = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, window=W)
+    assert (got - _band_sdpa_prefill(x, W)).abs().max() < 1e-12
+
+
+def test_prefill_window_limits():
+    x = gi.prefill_inputs(1, 30, 4, 2, 8, torch.float32, seed=23)
+    full = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale)
+    assert torch.equal(oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, window=30), full)
+    assert torch.equal(oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, window=1000), full)
+    one = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, window=1)
+    for i in range(4):                       # W = 1: every query sees only itself
+        assert torch.equal(one[0, :, i], x.v[0, :, i // 2].double())
+
+
+def test_decode_window_is_decode_on_the_last_W_positions():
+    x = gi.decode_inputs(3, 8, 2, 16, 50, torch.bfloat16, seed=24, seqlens=[50, 7, 23])
+    W = 10
+    got = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, window=W)
+    for b, T in enumerate([50, 7, 23]):
+        lo = max(0, T - W)
+        ref = oracle.gqa_decode(x.q[b:b + 1], x.k_cache[b:b + 1, :, lo:T], x.v_cache[b:b + 1, :, lo:T],
+                                [T - lo], x.scale)
+        assert torch.equal(got[b], ref[0])
+    assert torch.equal(oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, window=50),
+                       oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale))
