@@ -40,7 +40,8 @@ ROW_WORKLOADS = ["tiny_decode_fp32", "llama2_70b_ragged_decode"] + \
     ["long_ctx_decode_G%d" % g for g in (1, 2, 4, 8, 16, 32)] + ["causal_prefill", "meanpool_init",
                                                                 "qkv_append_llama2_7b",
                                                                 "causal_prefill_window4096",
-                                                                "llama2_70b_ragged_decode_window4096"]
+                                                                "llama2_70b_ragged_decode_window4096",
+                                                                "layer_decode_llama2_7b"]
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, bytes, from ncu
 # captures of the current kernels (profiles/*.md); a workload missing here has
@@ -411,9 +412,46 @@ class QkvAppend:
                 "sample": "the projections and append of sequence 0 of %d" % x.B}
 
 
+class LayerDecode(QkvAppend):
+    """One decode step of the attention layer: append, attend over the cache, W_O."""
+    kind = "layer"
+
+    def __init__(self, name, gqa, device="cuda"):
+        super().__init__(name, gqa, device)
+        x = self.x
+        gen = torch.Generator().manual_seed(1)
+        D = x.H * x.d_h
+        self.wo = (torch.randn(D, x.d, generator=gen) * D ** -0.5).to(x.h.dtype).to(device)
+        self.out = torch.empty((x.B, x.d), dtype=x.h.dtype, device=device)
+        self.ws = torch.empty(int(gqa.lib.gqa_layer_decode_workspace_bytes(x.B, x.H, x.G, x.d_h,
+                                                                             x.T_cap, gqa.GQA_BF16)),
+                              dtype=torch.uint8, device=device)
+        e = x.h.element_size()
+        T_after = (x.seqlens.clamp(max=x.T_cap - 1) + 1).sum().item()
+        # weights (Q, K, V, O) once, the cache over the lengths after the append, small tensors
+        self.bytes = ((x.d * (x.H + 2 * x.G) * x.d_h + D * x.d) + 2 * T_after * x.G * x.d_h
+                      + x.B * x.d * 2 + 2 * x.B * x.H * x.d_h + 2 * x.B * x.G * x.d_h) * e
+        self.launches_per_step = 2 * ((x.B + 31) // 32) + 2
+
+    def step(self, stream=None):
+        self.gqa.layer_decode_step(self.h, self.wq, self.wk, self.wv, self.wo, self.kc, self.vc,
+                                   self.sl, out=self.out, seqlens_out=self.sl_out,
+                                   workspace=self.ws, stream=stream)
+
+    def oracle_sample(self, budget_s):
+        import oracle
+        x = self.x
+        t0 = time.perf_counter()
+        oracle.layer_decode_step(x.h[:1], x.W_Q, x.W_K, x.W_V, self.wo.cpu(), x.k_cache[:1],
+                                 x.v_cache[:1], x.seqlens[:1], x.d_h ** -0.5)
+        return {"seconds": time.perf_counter() - t0, "fraction_of_step": 1.0 / x.B,
+                "sample": "the whole layer step of sequence 0 of %d" % x.B}
+
+
 def make(name, gqa):
     kind = gi.WORKLOADS[name]["kind"]
-    return {"decode": Decode, "prefill": Prefill, "meanpool": MeanPool, "qkv": QkvAppend}[kind](name, gqa)
+    return {"decode": Decode, "prefill": Prefill, "meanpool": MeanPool, "qkv": QkvAppend,
+            "layer": LayerDecode}[kind](name, gqa)
 
 
 # ------------------------------------------------------------------ timing
@@ -532,7 +570,8 @@ def run_reference(args, world, rank):
 def make_host_only(name):
     """A workload object with host inputs only (the reference arm needs no GPU)."""
     kind = gi.WORKLOADS[name]["kind"]
-    cls = {"decode": Decode, "prefill": Prefill, "meanpool": MeanPool, "qkv": QkvAppend}[kind]
+    cls = {"decode": Decode, "prefill": Prefill, "meanpool": MeanPool, "qkv": QkvAppend,
+           "layer": QkvAppend}[kind]
     obj = cls.__new__(cls)
     w = gi.WORKLOADS[name]
     obj.name, obj.w, obj.gqa = name, w, None
@@ -551,7 +590,7 @@ def make_host_only(name):
         obj.x = x
         Wn = obj.window if obj.window else x.S
         obj.flops = 4 * x.B * x.H * x.d_h * sum(min(s + 1, Wn) for s in range(x.S))
-    elif kind == "qkv":
+    elif kind in ("qkv", "layer"):
         x = gi.qkv_inputs(w["B"], w["d"], w["H"], w["G"], w["d_h"], w["T"], w["dtype"], seed=0)
         obj.x = x
         obj.bytes = (x.d * (x.H + 2 * x.G) * x.d_h + x.B * x.d + x.B * x.H * x.d_h

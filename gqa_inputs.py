@@ -38,6 +38,9 @@ WORKLOADS = {
     # one decode token's projections + cache append, Llama-2-7B shape (d = 4096)
     "qkv_append_llama2_7b": dict(kind="qkv", B=16, d=4096, H=32, G=8, d_h=128, T=4096,
                                  dtype=torch.bfloat16),
+    # one decode step of the whole attention layer (append, attend, W_O), same shape
+    "layer_decode_llama2_7b": dict(kind="layer", B=16, d=4096, H=32, G=8, d_h=128, T=4096,
+                                   dtype=torch.bfloat16),
     # half-length prefill (150 MB of q/k/v/out, above the 126 MB L2) for profiler captures
     "causal_prefill_profile": dict(kind="prefill", B=1, S=4096, H=64, G=8, d_h=128,
                                    dtype=torch.bfloat16),
@@ -182,6 +185,6 @@ def workload_inputs(name, seed=0):
                              ragged=w["ragged"])
     if w["kind"] == "prefill":
         return prefill_inputs(w["B"], w["S"], w["H"], w["G"], w["d_h"], w["dtype"], seed)
-    if w["kind"] == "qkv":
+    if w["kind"] in ("qkv", "layer"):
         return qkv_inputs(w["B"], w["d"], w["H"], w["G"], w["d_h"], w["T"], w["dtype"], seed)
     return meanpool_inputs(w["H"], w["d_h"], w["d"], w["dtype"], seed, w["std"])

@@ -229,6 +229,64 @@ GQA_API int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, cons
                            gqa_dtype dt, gqa_stream_t stream);
 
 /*
+ * gqa_init_kv_heads -- the mean-pool initialisation and the two alternatives
+ * the pages set against it, selected by `mode`:
+ *   GQA_INIT_MEAN      the group mean, identical to gqa_meanpool_kv;
+ *   GQA_INIT_SELECT    WK_out[g] = WK[g*r + select], picking one head of each
+ *                      group ("Grouped-Query Attention", llm-arch-kb, section 2
+ *                      "Uptraining recipe", the alternative reported worse than
+ *                      averaging); an exact copy;
+ *   GQA_INIT_WEIGHTED  WK_out[g] = sum_j wK[g*r + j] * WK[g*r + j] (same for V
+ *                      with wV), a weighted average over the group's heads with
+ *                      caller-given weights (section 4, weighted grouped-query
+ *                      attention); binary64 products and sums in ascending head
+ *                      order, one nearest-even rounding, bit-exact with that
+ *                      definition.
+ *   head_weights  device, [2, H] float: wK then wV (mode GQA_INIT_WEIGHTED only)
+ *   select        0 <= select < H/G (mode GQA_INIT_SELECT only)
+ * Other arguments and limits as gqa_meanpool_kv.
+ */
+enum { GQA_INIT_MEAN = 0, GQA_INIT_SELECT = 1, GQA_INIT_WEIGHTED = 2 };
+GQA_API int gqa_init_kv_heads(const void *WK, const void *WV, void *WK_out, void *WV_out,
+                              int H, int G, int d_h, int d, int mode,
+                              const float *head_weights, int select, gqa_dtype dt,
+                              gqa_stream_t stream);
+
+/*
+ * gqa_out_project -- the output projection of the attention block, the
+ * concatenated heads times W_O ("Grouped-Query Attention", llm-arch-kb,
+ * section 2: the outputs concatenate across heads and are projected by W_O;
+ * section 3: o.reshape(B, T, H*d_h) @ W_O), for one token per sequence:
+ *     out[b, :] = x[b, :] W                 x [B, K], W [K, N], out [B, N]
+ * bf16 in, fp32 accumulation, one rounding to bf16.  Same skinny-GEMM kernel
+ * as gqa_qkv_append.  Supported: bf16, K a multiple of 128, N of 64; x and W
+ * 16-byte aligned.
+ */
+GQA_API int gqa_out_project(const void *x, const void *W, void *out, int B, int K, int N,
+                            gqa_dtype dt, gqa_stream_t stream);
+
+/*
+ * gqa_layer_decode_step -- one decode step of a whole GQA attention layer
+ * (section 3's gqa() for one new token per sequence): gqa_qkv_append (q, and
+ * k/v appended at seqlens[b]), then gqa_decode_window over seqlens_out
+ * (which includes the new token), then gqa_out_project of the attention
+ * output with W_O into out [B, d].  q and the attention output are kept in
+ * bf16 in the workspace between the steps.
+ *   W_O          device, [H*d_h, d] bf16
+ *   seqlens_out  required: the lengths after the append
+ *   workspace    >= gqa_layer_decode_workspace_bytes(...), 256-byte aligned
+ * Other arguments as gqa_qkv_append and gqa_decode_window (window 0 = full).
+ */
+GQA_API size_t gqa_layer_decode_workspace_bytes(int B, int H, int G, int d_h, int T_cap,
+                                                gqa_dtype dt);
+GQA_API int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_K,
+                                  const void *W_V, const void *W_O, void *k_cache,
+                                  void *v_cache, const int32_t *seqlens, int32_t *seqlens_out,
+                                  float scale, int window, void *out, int B, int d, int H, int G,
+                                  int d_h, int T_cap, gqa_dtype dt, void *workspace,
+                                  size_t workspace_bytes, gqa_stream_t stream);
+
+/*
  * gqa_get_status -- synchronises `stream`, then reads and clears the device
  * status word: GQA_OK, GQA_ERR_SEQLEN or GQA_ERR_TIMEOUT (device-side
  * conditions of earlier calls on this device), or GQA_ERR_CUDA if the

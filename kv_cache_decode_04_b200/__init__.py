@@ -23,7 +23,7 @@ import os
 import torch
 
 __all__ = ["decode", "decode_noalloc", "decode_workspace_bytes", "prefill_causal", "meanpool_kv",
-           "qkv_append",
+           "qkv_append", "init_kv_heads", "out_project", "layer_decode_step",
            "kv_cache_bytes", "get_status", "GQAError", "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqa.so")
@@ -35,8 +35,9 @@ _ERRORS = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGN", -4: "CUDA", -5: "WORKS
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_kv_cache_bytes", "gqa_decode_workspace_bytes", "gqa_decode",
            "gqa_decode_window", "gqa_decode_noalloc", "gqa_prefill_causal",
-           "gqa_prefill_causal_window", "gqa_meanpool_kv", "gqa_qkv_append", "gqa_get_status",
-           "gqa_last_error_string", "gqa_version")
+           "gqa_prefill_causal_window", "gqa_meanpool_kv", "gqa_init_kv_heads", "gqa_qkv_append",
+           "gqa_out_project", "gqa_layer_decode_workspace_bytes", "gqa_layer_decode_step",
+           "gqa_get_status", "gqa_last_error_string", "gqa_version")
 
 
 class GQAError(RuntimeError):
@@ -72,6 +73,15 @@ def _load():
     L.gqa_qkv_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                  i32, vp]
     L.gqa_qkv_append.restype = i32
+    L.gqa_init_kv_heads.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, i32, i32, vp]
+    L.gqa_init_kv_heads.restype = i32
+    L.gqa_out_project.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+    L.gqa_out_project.restype = i32
+    L.gqa_layer_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.gqa_layer_decode_workspace_bytes.restype = sz
+    L.gqa_layer_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, f32, i32, vp, i32, i32,
+                                        i32, i32, i32, i32, i32, vp, sz, vp]
+    L.gqa_layer_decode_step.restype = i32
     L.gqa_get_status.argtypes = [vp]
     L.gqa_get_status.restype = i32
     L.gqa_last_error_string.argtypes = []
@@ -217,6 +227,35 @@ def meanpool_kv(wk, wv, G, out_k=None, out_v=None, stream=None):
     return out_k, out_v
 
 
+GQA_INIT_MEAN, GQA_INIT_SELECT, GQA_INIT_WEIGHTED = 0, 1, 2
+
+
+def init_kv_heads(wk, wv, G, mode="mean", head_weights=None, select=0, out_k=None, out_v=None,
+                  stream=None):
+    """G K/V heads from H MHA heads: mode "mean" (= meanpool_kv), "select" (head
+    `select` of each group) or "weighted" (head_weights [2, H] device float32:
+    K's weights then V's)."""
+    H, d_h, d = wk.shape
+    if tuple(wv.shape) != tuple(wk.shape) or wk.dtype != wv.dtype:
+        raise ValueError("WK and WV must have the same shape and dtype")
+    m = {"mean": GQA_INIT_MEAN, "select": GQA_INIT_SELECT, "weighted": GQA_INIT_WEIGHTED}[mode]
+    code = _dtype_code(wk)
+    if out_k is None:
+        out_k = torch.empty((G, d_h, d), dtype=wk.dtype, device=wk.device)
+    if out_v is None:
+        out_v = torch.empty((G, d_h, d), dtype=wk.dtype, device=wk.device)
+    wp = None
+    if head_weights is not None:
+        if head_weights.dtype != torch.float32 or head_weights.numel() != 2 * H:
+            raise ValueError("head_weights must be float32 [2, H]")
+        wp = _dev(head_weights, "head_weights")
+    rc = lib.gqa_init_kv_heads(_dev(wk, "WK"), _dev(wv, "WV"), _dev(out_k, "WK_out"),
+                               _dev(out_v, "WV_out"), H, int(G), d_h, d, m, wp, int(select), code,
+                               _stream(stream))
+    _check(rc)
+    return out_k, out_v
+
+
 def qkv_append(h, W_Q, W_K, W_V, k_cache, v_cache, seqlens, q_out=None, seqlens_out=None,
                stream=None):
     """One decode token: q = h W_Q, and h W_K, h W_V appended to the KV cache.
@@ -242,6 +281,50 @@ def qkv_append(h, W_Q, W_K, W_V, k_cache, v_cache, seqlens, q_out=None, seqlens_
                             d_h, T_cap, code, _stream(stream))
     _check(rc)
     return q_out, seqlens_out
+
+
+def out_project(x, W, out=None, stream=None):
+    """out = x W for x [B, K] (e.g. the concatenated heads [B, H*d_h]) and W [K, N]."""
+    x2 = x.reshape(x.shape[0], -1)
+    B, K = x2.shape
+    if W.shape[0] != K:
+        raise ValueError("x and W disagree on K")
+    N = W.shape[1]
+    if out is None:
+        out = torch.empty((B, N), dtype=x.dtype, device=x.device)
+    _check(lib.gqa_out_project(_dev(x2, "x"), _dev(W, "W"), _dev(out, "out"), B, K, N,
+                               _dtype_code(x), _stream(stream)))
+    return out
+
+
+def layer_decode_step(h, W_Q, W_K, W_V, W_O, k_cache, v_cache, seqlens, scale=None, window=0,
+                      out=None, seqlens_out=None, workspace=None, stream=None):
+    """One decode step of the attention layer: append, attend, project.
+
+    Returns (out [B, d], seqlens_out)."""
+    B, d = h.shape
+    _, G, T_cap, d_h = k_cache.shape
+    H = W_Q.shape[1] // d_h
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_h)
+    if out is None:
+        out = torch.empty((B, d), dtype=h.dtype, device=h.device)
+    if seqlens_out is None:
+        seqlens_out = torch.empty_like(seqlens)
+    code = _dtype_code(h)
+    if workspace is None:
+        n = int(lib.gqa_layer_decode_workspace_bytes(B, H, G, d_h, T_cap, code))
+        if n == 0:
+            raise GQAError(-1, lib.gqa_last_error_string().decode())
+        workspace = torch.empty(n, dtype=torch.uint8, device=h.device)
+    rc = lib.gqa_layer_decode_step(_dev(h, "h"), _dev(W_Q, "W_Q"), _dev(W_K, "W_K"), _dev(W_V, "W_V"),
+                                   _dev(W_O, "W_O"), _dev(k_cache, "k_cache"),
+                                   _dev(v_cache, "v_cache"), _dev(seqlens, "seqlens"),
+                                   _dev(seqlens_out, "seqlens_out"), float(scale), int(window),
+                                   _dev(out, "out"), B, d, H, G, d_h, T_cap, code,
+                                   _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    _check(rc)
+    return out, seqlens_out
 
 
 def get_status(stream=None):

@@ -306,9 +306,15 @@ int gqa_prefill_causal_window(const void *q, const void *k, const void *v, void 
     return prefill_impl(q, k, v, out, B, S, H, G, d_h, scale, window, dt, stream);
 }
 
-int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *WV_out, int H, int G, int d_h,
-                    int d, gqa_dtype dt, gqa_stream_t stream) {
+static int init_heads_impl(const void *WK, const void *WV, void *WK_out, void *WV_out, int H, int G, int d_h,
+                           int d, int mode, const float *weights, int select, gqa_dtype dt, gqa_stream_t stream) {
     t_err[0] = 0;
+    if (mode != GQA_INIT_MEAN && mode != GQA_INIT_SELECT && mode != GQA_INIT_WEIGHTED)
+        return fail(GQA_ERR_INVALID, "unknown init mode %d", mode);
+    if (mode == GQA_INIT_SELECT && (G <= 0 || H % G != 0 || select < 0 || select >= H / G))
+        return fail(GQA_ERR_INVALID, "select must index a head inside its group (0 <= select < H/G)");
+    if (mode == GQA_INIT_WEIGHTED && (!weights || misaligned(weights, 4)))
+        return fail(GQA_ERR_INVALID, "weighted init needs 2*H device float weights");
     if (H <= 0 || G <= 0 || d_h <= 0 || d <= 0)
         return fail(GQA_ERR_INVALID, "dimensions must be positive (H=%d G=%d d_h=%d d=%d)", H, G, d_h, d);
     if (H % G != 0) return fail(GQA_ERR_INVALID, "G=%d must divide H=%d", G, H);
@@ -331,10 +337,21 @@ int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *WV_out, 
     DeviceInfo *d_ = nullptr;
     int rc = device_info(&d_);
     if (rc) return rc;
-    cudaError_t e = gqa::launch_meanpool(WK, WV, WK_out, WV_out, H, G, n, dt, d_->num_sms,
-                                         reinterpret_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return fail_cuda(e, "meanpool launch");
+    cudaError_t e = gqa::launch_init_heads(WK, WV, WK_out, WV_out, H, G, n, dt, mode, weights, select,
+                                           d_->num_sms, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "init-heads launch");
     return GQA_OK;
+}
+
+int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *WV_out, int H, int G, int d_h,
+                    int d, gqa_dtype dt, gqa_stream_t stream) {
+    return init_heads_impl(WK, WV, WK_out, WV_out, H, G, d_h, d, GQA_INIT_MEAN, nullptr, 0, dt, stream);
+}
+
+int gqa_init_kv_heads(const void *WK, const void *WV, void *WK_out, void *WV_out, int H, int G, int d_h,
+                      int d, int mode, const float *head_weights, int select, gqa_dtype dt,
+                      gqa_stream_t stream) {
+    return init_heads_impl(WK, WV, WK_out, WV_out, H, G, d_h, d, mode, head_weights, select, dt, stream);
 }
 
 int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V, void *q_out,
@@ -402,6 +419,76 @@ int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *
     cudaError_t e = gqa::launch_qkv_append(a, &tq, &tk, &tv, &th, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "qkv_append launch");
     return GQA_OK;
+}
+
+int gqa_out_project(const void *x, const void *W, void *out, int B, int K, int N, gqa_dtype dt,
+                    gqa_stream_t stream) {
+    t_err[0] = 0;
+    if (B <= 0 || K <= 0 || N <= 0) return fail(GQA_ERR_INVALID, "B, K and N must be positive");
+    if (!x || !W || !out) return fail(GQA_ERR_INVALID, "null tensor pointer");
+    if (dt != GQA_BF16) return fail(GQA_ERR_UNSUPPORTED, "out_project supports bf16 only");
+    if (K % 128 != 0 || N % 64 != 0)
+        return fail(GQA_ERR_UNSUPPORTED, "K must be a multiple of 128 and N of 64 (K=%d N=%d)", K, N);
+    if (misaligned(x, 16) || misaligned(W, 16) || misaligned(out, 2))
+        return fail(GQA_ERR_ALIGN, "x and W must be 16-byte aligned");
+    DeviceInfo *dev = nullptr;
+    int rc = device_info(&dev);
+    if (rc) return rc;
+    CUtensorMap tw, tx;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)K};
+        const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+        const cuuint32_t box[2] = {64, 128};
+        rc = make_tmap_bf16(&tw, W, 2, dims, strides, box);
+        if (rc) return rc;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)B};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {64, 32};
+        rc = make_tmap_bf16(&tx, x, 2, dims, strides, box);
+        if (rc) return rc;
+    }
+    cudaError_t e = gqa::launch_out_project(x, out, B, K, N, dev->status, wait_timeout_ns(), &tw, &tx,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "out_project launch");
+    return GQA_OK;
+}
+
+static size_t align256_host(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t gqa_layer_decode_workspace_bytes(int B, int H, int G, int d_h, int T_cap, gqa_dtype dt) {
+    const size_t dec = gqa_decode_workspace_bytes(B, H, G, d_h, T_cap, dt);
+    if (!dec) return 0;
+    return 2 * align256_host((size_t)B * H * d_h * 2) + dec;
+}
+
+int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_K, const void *W_V, const void *W_O,
+                          void *k_cache, void *v_cache, const int32_t *seqlens, int32_t *seqlens_out,
+                          float scale, int window, void *out, int B, int d, int H, int G, int d_h, int T_cap,
+                          gqa_dtype dt, void *workspace, size_t workspace_bytes, gqa_stream_t stream) {
+    t_err[0] = 0;
+    if (!seqlens_out) return fail(GQA_ERR_INVALID, "the layer step needs seqlens_out (lengths after the append)");
+    const size_t need = gqa_layer_decode_workspace_bytes(B, H, G, d_h, T_cap, dt);
+    if (!need) return decode_impl(nullptr, nullptr, nullptr, nullptr, scale, nullptr, B, H, G, d_h, T_cap, window, dt,
+                                  nullptr, 0, stream);
+    if (!workspace || workspace_bytes < need)
+        return fail(GQA_ERR_WORKSPACE, "layer workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (misaligned(workspace, 256)) return fail(GQA_ERR_ALIGN, "workspace must be 256-byte aligned");
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t qbytes = align256_host((size_t)B * H * d_h * 2);
+    void *q = ws, *attn = ws + qbytes;
+    // 1. q = h W_Q; k, v appended at seqlens[b]
+    int rc = gqa_qkv_append(h, W_Q, W_K, W_V, q, k_cache, v_cache, seqlens, seqlens_out, B, d, H, G, d_h, T_cap,
+                            dt, stream);
+    if (rc) return rc;
+    // 2. attention over the cache including the new token
+    rc = decode_impl(q, k_cache, v_cache, seqlens_out, scale, attn, B, H, G, d_h, T_cap, window, dt,
+                     ws + 2 * qbytes, workspace_bytes - 2 * qbytes, stream);
+    if (rc) return rc;
+    // 3. concatenated heads times W_O
+    return gqa_out_project(attn, W_O, out, B, H * d_h, d, dt, stream);
 }
 
 int gqa_get_status(gqa_stream_t stream) {

@@ -69,11 +69,19 @@ struct QkvArgs {
 cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUtensorMap *tk,
                               const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t stream);
 
+cudaError_t launch_out_project(const void *x, void *out, int B, int K, int N, unsigned *status,
+                               uint64_t timeout_ns, const CUtensorMap *tw, const CUtensorMap *tx,
+                               cudaStream_t stream);
+
 // Records `msg` as the calling thread's last error and returns `code`.
 int set_error(int code, const char *msg);
 
-// Mean-pool init.
+// Mean-pool init, and its select-one-head / weighted-average alternatives
+// (mode 0, 1, 2; weights [2H] device floats for mode 2, K's then V's).
 cudaError_t launch_meanpool(const void *wk, const void *wv, void *ok, void *ov, int H, int G,
                             long long n, int dtype, int num_sms, cudaStream_t stream);
+cudaError_t launch_init_heads(const void *wk, const void *wv, void *ok, void *ov, int H, int G,
+                              long long n, int dtype, int mode, const float *weights, int select,
+                              int num_sms, cudaStream_t stream);
 
 }  // namespace gqa

@@ -46,7 +46,8 @@ struct ProjParams {
     unsigned *status;
     int B, d, H, G, d_h, T_cap;
     int b0;                   // first sequence of this launch
-    int nq, nk;               // 64-column blocks of W_Q and of W_K (= of W_V)
+    int nq, nk;               // 64-column blocks of W_Q and of W_K (= of W_V); nk = 0: one weight
+    int out_ld;               // row stride of q_out (H*d_h, or N for a single weight)
     unsigned long long timeout_ns;
 };
 
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         const __nv_bfloat16 o = __float2bfloat16_rn(v);
         const int n = col0 + c;
         if (region == 0) {
-            p.q_out[(size_t)b * p.H * p.d_h + n] = o;
+            p.q_out[(size_t)b * p.out_ld + n] = o;
         } else {
             const int T = p.seqlens[b];
             if (T < 0 || T >= p.T_cap) {
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             cache[(((size_t)b * p.G + g) * p.T_cap + T) * p.d_h + dim] = o;
         }
     }
-    if (cb == 0 && p.seqlens_out)
+    if (cb == 0 && p.nk > 0 && p.seqlens_out)
         for (int b = p.b0 + tid; b < min(p.B, p.b0 + RB * 16); b += kCW * 32) {
             const int T = p.seqlens[b];
             p.seqlens_out[b] = (T >= 0 && T < p.T_cap) ? T + 1 : T;
@@ -240,11 +241,34 @@ cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUt
     p.T_cap = a.T_cap;
     p.nq = a.H * a.d_h / kNT;
     p.nk = a.G * a.d_h / kNT;
+    p.out_ld = a.H * a.d_h;
     p.timeout_ns = a.timeout_ns;
     for (int b0 = 0; b0 < a.B; b0 += 32) {  // 32 sequences per launch
         p.b0 = b0;
         const cudaError_t e =
             (a.B - b0 > 16) ? run_proj<2>(p, tq, tk, tv, th, st) : run_proj<1>(p, tq, tk, tv, th, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+// out[B, N] = x[B, K] W[K, N]: the same kernel with one weight and no cache.
+cudaError_t launch_out_project(const void *x, void *out, int B, int K, int N, unsigned *status,
+                               uint64_t timeout_ns, const CUtensorMap *tw, const CUtensorMap *tx,
+                               cudaStream_t st) {
+    ProjParams p = {};
+    p.h = static_cast<const __nv_bfloat16 *>(x);
+    p.q_out = static_cast<__nv_bfloat16 *>(out);
+    p.status = status;
+    p.B = B;
+    p.d = K;
+    p.nq = N / kNT;
+    p.nk = 0;
+    p.out_ld = N;
+    p.timeout_ns = timeout_ns;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+        p.b0 = b0;
+        const cudaError_t e = (B - b0 > 16) ? run_proj<2>(p, tw, tw, tw, tx, st) : run_proj<1>(p, tw, tw, tw, tx, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -75,6 +75,8 @@ def _load():
     lib.oracle_gqa_prefill_causal.restype = i32
     lib.oracle_meanpool.argtypes = [vp, i32, i32, i32, ctypes.c_size_t, vp]
     lib.oracle_meanpool.restype = i32
+    lib.oracle_init_heads.argtypes = [vp, i32, i32, i32, ctypes.c_size_t, i32, vp, i32, vp]
+    lib.oracle_init_heads.restype = i32
     lib.oracle_project.argtypes = [vp, i32, vp, i32, vp, i32, i32, i32]
     lib.oracle_project.restype = i32
     lib.oracle_round_bf16.argtypes = [vp, vp, ctypes.c_size_t]
@@ -280,3 +282,42 @@ def qkv_append(h, W_Q, W_K, W_V, k_cache, v_cache, seqlens):
             sl[b] = t + 1
             appended[b] = True
     return q, k, v, kc, vc, sl.to(torch.int32), appended
+
+
+def init_heads(W, G, mode, weights=None, select=0, out_dtype=None):
+    """Alternatives to the mean-pool init, rounded once to out_dtype.
+
+    mode "select": head `select` of each group; mode "weighted": sum of the
+    group's heads times caller weights [H] (binary64, ascending head order).
+    """
+    lib = _load()
+    wt, wp, wdt = _as_host(W)
+    H = wt.shape[0]
+    n = wt[0].numel() if H else 0
+    out = torch.empty((G,) + tuple(wt.shape[1:]), dtype=torch.float64)
+    m = {"select": 1, "weighted": 2}[mode]
+    wts = torch.as_tensor(weights if weights is not None else [0.0] * H,
+                          dtype=torch.float64).reshape(-1).contiguous()
+    if wts.numel() != H:
+        raise ValueError("need one weight per head")
+    rc = lib.oracle_init_heads(wp, wdt, H, int(G), n, m, wts.data_ptr(), int(select), out.data_ptr())
+    if rc != 0:
+        raise ValueError("oracle_init_heads failed (rc=%d)" % rc)
+    return round_to(out, out_dtype or W.dtype)
+
+
+def layer_decode_step(h, W_Q, W_K, W_V, W_O, k_cache, v_cache, seqlens, scale, window=0):
+    """One decode step of the attention layer ("Grouped-Query Attention",
+    section 3's gqa() for one token): project and append (qkv_append), attend
+    over the lengths after the append (gqa_decode), then the concatenated heads
+    times W_O.  Values stored in bf16 between the steps are rounded to bf16 here
+    at the same points: q, the appended k/v rows (the cache is bf16) and the
+    attention output.  Returns (out float64 [B, d], seqlens_after)."""
+    q, k, v, kc, vc, sl, app = qkv_append(h, W_Q, W_K, W_V, k_cache, v_cache, seqlens)
+    st = torch.bfloat16
+    qs = round_to(q, st)
+    kcs, vcs = round_to(kc, st), round_to(vc, st)
+    attn = gqa_decode(qs, kcs, vcs, sl, scale, window=window)
+    B, H, d_h = attn.shape
+    attn_s = round_to(attn, st).reshape(B, H * d_h)
+    return project(attn_s, W_O), sl

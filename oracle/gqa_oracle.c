@@ -344,3 +344,39 @@ int oracle_project(const void *h, int h_dt, const void *W, int w_dt, double *out
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* other initialisations of the G heads from the H MHA heads           */
+/* ------------------------------------------------------------------ */
+
+/* mode 1: out[g] = W[g*r + sel] -- picking one head per group, the first
+ *         alternative the GQA paper compares with averaging ("Grouped-Query
+ *         Attention", section 2, "Uptraining recipe");
+ * mode 2: out[g] = sum_{i: g(i)=g} w[i] * W[i], ascending i, binary64 products
+ *         and sums -- a weighted average over the heads of a group with
+ *         caller-given weights (section 4, weighted grouped-query attention).
+ * W [H, n]; out [G, n] in binary64 (rounded by the caller). */
+int oracle_init_heads(const void *W, int dt, int H, int G, size_t n, int mode, const double *w,
+                      int sel, double *out) {
+    if (G <= 0 || H % G != 0) return -1;
+    const int r = H / G;
+    if (mode == 1) {
+        if (sel < 0 || sel >= r) return -1;
+        for (int i = 0; i < H; ++i) {
+            int g = oracle_group_of_head(i, H, G);
+            if (i - g * r != sel) continue; /* the head's position inside its group */
+            for (size_t e = 0; e < n; ++e) out[(size_t)g * n + e] = ld(W, dt, (size_t)i * n + e);
+        }
+        return 0;
+    }
+    if (mode == 2) {
+        memset(out, 0, sizeof(double) * (size_t)G * n);
+        for (int i = 0; i < H; ++i) {
+            int g = oracle_group_of_head(i, H, G);
+            for (size_t e = 0; e < n; ++e)
+                out[(size_t)g * n + e] += w[i] * ld(W, dt, (size_t)i * n + e);
+        }
+        return 0;
+    }
+    return -1;
+}

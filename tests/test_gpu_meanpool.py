@@ -60,3 +60,34 @@ def test_meanpool_unaligned_views(gqa):
     gqa.get_status()
     assert torch.equal(bits(ok.cpu()), bits(oracle.meanpool(wk.cpu(), G)))
     assert torch.equal(bits(ov.cpu()), bits(oracle.meanpool(wv.cpu(), G)))
+
+
+# ------------------------------------------------------------ the alternatives to the mean
+
+@pytest.mark.parametrize("H,G,d_h,d", [(64, 8, 128, 64), (12, 4, 3, 5), (16, 1, 8, 24)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_init_select_and_weighted_bit_exact(gqa, H, G, d_h, d, dtype):
+    wk, wv = gi.meanpool_inputs(H, d_h, d, dtype=dtype, seed=H + 3 * d, std=0.5)
+    r = H // G
+    for sel in sorted({0, r - 1}):
+        ok, ov = gqa.init_kv_heads(wk.cuda(), wv.cuda(), G, mode="select", select=sel)
+        gqa.get_status()
+        assert torch.equal(bits(ok.cpu()), bits(oracle.init_heads(wk, G, "select", select=sel)))
+        assert torch.equal(bits(ov.cpu()), bits(oracle.init_heads(wv, G, "select", select=sel)))
+    w = torch.rand(2, H, generator=torch.Generator().manual_seed(H)) + 0.1
+    ok, ov = gqa.init_kv_heads(wk.cuda(), wv.cuda(), G, mode="weighted", head_weights=w.cuda())
+    gqa.get_status()
+    assert torch.equal(bits(ok.cpu()), bits(oracle.init_heads(wk, G, "weighted", weights=w[0].double())))
+    assert torch.equal(bits(ov.cpu()), bits(oracle.init_heads(wv, G, "weighted", weights=w[1].double())))
+    # the mean through the same entry point equals gqa_meanpool_kv's
+    ok, ov = gqa.init_kv_heads(wk.cuda(), wv.cuda(), G, mode="mean")
+    gqa.get_status()
+    assert torch.equal(bits(ok.cpu()), bits(oracle.meanpool(wk, G)))
+
+
+def test_init_rejects_bad_selection(gqa):
+    wk, wv = gi.meanpool_inputs(8, 4, 8, seed=1)
+    with pytest.raises(gqa.GQAError):
+        gqa.init_kv_heads(wk.cuda(), wv.cuda(), 2, mode="select", select=4)
+    with pytest.raises(gqa.GQAError):
+        gqa.init_kv_heads(wk.cuda(), wv.cuda(), 2, mode="weighted")

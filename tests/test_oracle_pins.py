@@ -455,3 +455,49 @@ def test_decode_window_is_decode_on_the_last_W_positions():
         assert torch.equal(got[b], ref[0])
     assert torch.equal(oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, window=50),
                        oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale))
+
+
+# ----------------------------------------------------------------- init variants
+
+def test_init_select_picks_one_head_per_group():
+    """KB s2: the alternative of picking a single head from each group."""
+    wk, _ = gi.meanpool_inputs(16, 4, 8, seed=25)
+    for sel in range(4):
+        got = oracle.init_heads(wk, 4, "select", select=sel)
+        assert torch.equal(got.view(torch.int16), wk[sel::4].view(torch.int16))
+
+
+def test_init_weighted_special_cases():
+    """Weighted averaging (KB s4): 1/r weights give the mean (exact for r a power
+    of two), one-hot weights give selection, doubling the weights doubles the result."""
+    wk, _ = gi.meanpool_inputs(16, 4, 8, seed=26, std=0.5)
+    H, G, r = 16, 4, 4
+    mean = oracle.meanpool(wk, G)
+    assert torch.equal(oracle.init_heads(wk, G, "weighted", weights=[1 / r] * H).view(torch.int16),
+                       mean.view(torch.int16))
+    onehot = [1.0 if i % r == 2 else 0.0 for i in range(H)]
+    assert torch.equal(oracle.init_heads(wk, G, "weighted", weights=onehot).view(torch.int16),
+                       oracle.init_heads(wk, G, "select", select=2).view(torch.int16))
+    wts = torch.rand(H, generator=torch.Generator().manual_seed(27)).double()
+    a = oracle.init_heads(wk, G, "weighted", weights=wts, out_dtype=torch.float32)
+    b = oracle.init_heads(wk, G, "weighted", weights=2 * wts, out_dtype=torch.float32)
+    assert torch.equal(2 * a, b)
+    ref = torch.stack([sum(float(wts[g * r + j]) * wk[g * r + j].double() for j in range(r)) for g in range(G)])
+    assert (a.double() - ref).abs().max() < 1e-6
+
+
+def test_layer_step_with_identity_output_projection_is_the_attention():
+    """With W_O = I (d = H*d_h) the layer output is the attention output itself."""
+    H, G, d_h = 4, 2, 32
+    d = H * d_h
+    x = gi.qkv_inputs(2, d, H, G, d_h, 9, seed=28, seqlens=[3, 8])
+    eye = torch.eye(d, dtype=torch.bfloat16)
+    out, sl = oracle.layer_decode_step(x.h, x.W_Q, x.W_K, x.W_V, eye, x.k_cache, x.v_cache,
+                                       x.seqlens, d_h ** -0.5)
+    q, k, v, kc, vc, sl2, _ = oracle.qkv_append(x.h, x.W_Q, x.W_K, x.W_V, x.k_cache, x.v_cache,
+                                                x.seqlens)
+    st = torch.bfloat16
+    attn = oracle.gqa_decode(oracle.round_to(q, st), oracle.round_to(kc, st), oracle.round_to(vc, st),
+                             sl2, d_h ** -0.5)
+    assert torch.equal(out, oracle.round_to(attn, st).double().reshape(2, d))
+    assert sl.tolist() == [4, 9]
