@@ -294,6 +294,18 @@ GQA_API int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_
  */
 GQA_API int gqa_get_status(gqa_stream_t stream);
 
+/*
+ * gqa_selftest_wait_timeout -- checks the failure-detection path without
+ * hanging or faulting the GPU: one CTA waits, with the bounded wait every
+ * kernel here uses, on a barrier that nothing arrives at; after `limit_ns`
+ * nanoseconds (0 < limit_ns <= 1e10) it gives up, sets the GQA_ERR_TIMEOUT
+ * status bit and returns.  `waited` (device int, may be NULL) receives 1 if
+ * the wait ran out.  A following gqa_get_status returns GQA_ERR_TIMEOUT and
+ * the context stays usable.  (A host-side test hook; the pages have no
+ * counterpart.)
+ */
+GQA_API int gqa_selftest_wait_timeout(uint64_t limit_ns, int *waited, gqa_stream_t stream);
+
 /* Reason for the last non-OK return on the calling thread ("" if none). */
 GQA_API const char *gqa_last_error_string(void);
 

@@ -37,7 +37,7 @@ EXPORTS = ("gqa_kv_cache_bytes", "gqa_decode_workspace_bytes", "gqa_decode",
            "gqa_decode_window", "gqa_decode_noalloc", "gqa_prefill_causal",
            "gqa_prefill_causal_window", "gqa_meanpool_kv", "gqa_init_kv_heads", "gqa_qkv_append",
            "gqa_out_project", "gqa_layer_decode_workspace_bytes", "gqa_layer_decode_step",
-           "gqa_get_status", "gqa_last_error_string", "gqa_version")
+           "gqa_selftest_wait_timeout", "gqa_get_status", "gqa_last_error_string", "gqa_version")
 
 
 class GQAError(RuntimeError):
@@ -82,6 +82,8 @@ def _load():
     L.gqa_layer_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, f32, i32, vp, i32, i32,
                                         i32, i32, i32, i32, i32, vp, sz, vp]
     L.gqa_layer_decode_step.restype = i32
+    L.gqa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp]
+    L.gqa_selftest_wait_timeout.restype = i32
     L.gqa_get_status.argtypes = [vp]
     L.gqa_get_status.restype = i32
     L.gqa_last_error_string.argtypes = []

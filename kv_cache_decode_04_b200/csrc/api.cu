@@ -491,6 +491,20 @@ int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_K, const
     return gqa_out_project(attn, W_O, out, B, H * d_h, d, dt, stream);
 }
 
+int gqa_selftest_wait_timeout(uint64_t limit_ns, int *waited, gqa_stream_t stream) {
+    t_err[0] = 0;
+    if (limit_ns == 0 || limit_ns > 10000000000ull)
+        return fail(GQA_ERR_INVALID, "limit_ns must be in (0, 1e10]");
+    if (misaligned(waited, 4)) return fail(GQA_ERR_ALIGN, "waited must be 4-byte aligned");
+    DeviceInfo *dev = nullptr;
+    int rc = device_info(&dev);
+    if (rc) return rc;
+    cudaError_t e = gqa::launch_wait_timeout_selftest(dev->status, limit_ns, waited,
+                                                      reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "self-test launch");
+    return GQA_OK;
+}
+
 int gqa_get_status(gqa_stream_t stream) {
     t_err[0] = 0;
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

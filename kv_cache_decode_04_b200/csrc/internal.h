@@ -73,6 +73,10 @@ cudaError_t launch_out_project(const void *x, void *out, int B, int K, int N, un
                                uint64_t timeout_ns, const CUtensorMap *tw, const CUtensorMap *tx,
                                cudaStream_t stream);
 
+// One CTA waits on an mbarrier nothing arrives at, with the bounded wait.
+cudaError_t launch_wait_timeout_selftest(unsigned *status, uint64_t limit_ns, int *waited,
+                                         cudaStream_t stream);
+
 // Records `msg` as the calling thread's last error and returns `code`.
 int set_error(int code, const char *msg);
 
