@@ -22,9 +22,10 @@
 //   scale*log2(e), which leaves the result unchanged.
 //
 // bf16 path: a producer warp streams [64 x d_h] K and V tiles with TMA
-// (128-byte swizzle) through a 4-stage mbarrier ring; four consumer warps run
-// warp-level bf16 tensor-core MMAs (scores, then P.V with P rounded to bf16)
-// and an fp32 online softmax; query rows are padded to 16 per MMA tile.
+// (128-byte swizzle) through a 2-stage mbarrier ring (two CTAs per SM); four
+// consumer warps run warp-level bf16 tensor-core MMAs (scores, then P.V with P
+// rounded to bf16) and an fp32 online softmax; query rows are padded to 16 per
+// MMA tile.
 // fp32 path: CUDA-core fp32 arithmetic throughout (no TF32).
 #include <atomic>
 
@@ -166,7 +167,9 @@ __device__ __forceinline__ uint32_t swz(int tok, int dim) {
 
 // ----------------------------------------------------------------- bf16
 
-template <int D, int NMT>
+// RR: rows of the cross-slice reduction buffer per 16-row head tile (the
+// group's H/G heads when they are fewer than 16, so the buffer shrinks).
+template <int D, int NMT, int STAGES, int RR>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_split_bf16(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
@@ -176,22 +179,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     constexpr int NSL = kCWarps / NMT;  // token slices of a tile
     constexpr int TPS = kTile / NSL;    // tokens per slice
     constexpr int ROWF = D + 2;         // reduction row: m, l, o[D]
-    constexpr int RED_FLOATS = NSL > 1 ? NSL * NMT * 16 * ROWF : 0;
+    constexpr int RED_FLOATS = NSL > 1 ? NSL * NMT * RR * ROWF : 0;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint8_t *stages = smem;
-    float *red = reinterpret_cast<float *>(smem + kStages * STAGE_BYTES);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * STAGE_BYTES + RED_FLOATS * 4);
-    uint64_t *empty = full + kStages;
-    int *abort_flag = reinterpret_cast<int *>(empty + kStages);
+    float *red = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES + RED_FLOATS * 4);
+    uint64_t *empty = full + STAGES;
+    int *abort_flag = reinterpret_cast<int *>(empty + STAGES);
     int *cu = abort_flag + 1;
     int *scratch = cu + p.B + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kCWarps);
         }
@@ -219,8 +222,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             Cursor c;
             cursor_seek(cu, p.B, p.G, u_begin, c);
             for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
                 if (*vabort || !mbar_wait(&empty[s], ph ^ 1, p.timeout_ns)) {
                     set_status(p.status, STATUS_TIMEOUT);
                     *vabort = 1;
@@ -277,8 +280,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             m_a = m_b = -INFINITY;
             l_a = l_b = 0.f;
         }
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
         if (!dead && (*vabort || !mbar_wait(&full[s], ph, p.timeout_ns))) {
             dead = true;
             *vabort = 1;
@@ -430,20 +433,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 if (q4 == 0) p.ws_ml[rec * p.r + hl_b] = make_float2(m_b, lb);
             }
         } else {
-            float *ra = red + ((sl * NMT + mt) * 16 + g8) * ROWF;
+            // rows g8 and g8+8 of this warp's head tile; rows >= RR are past H/G
+            float *ra = red + ((sl * NMT + mt) * RR + g8) * ROWF;
             float *rb = ra + 8 * ROWF;
-            if (q4 == 0) {
-                ra[0] = m_a;
-                ra[1] = la;
-                rb[0] = m_b;
-                rb[1] = lb;
-            }
+            if (g8 < RR) {
+                if (q4 == 0) {
+                    ra[0] = m_a;
+                    ra[1] = la;
+                }
 #pragma unroll
-            for (int nn = 0; nn < D / 8; ++nn) {
-                ra[2 + nn * 8 + 2 * q4] = o[nn][0];
-                ra[3 + nn * 8 + 2 * q4] = o[nn][1];
-                rb[2 + nn * 8 + 2 * q4] = o[nn][2];
-                rb[3 + nn * 8 + 2 * q4] = o[nn][3];
+                for (int nn = 0; nn < D / 8; ++nn) {
+                    ra[2 + nn * 8 + 2 * q4] = o[nn][0];
+                    ra[3 + nn * 8 + 2 * q4] = o[nn][1];
+                }
+            }
+            if (g8 + 8 < RR) {
+                if (q4 == 0) {
+                    rb[0] = m_b;
+                    rb[1] = lb;
+                }
+#pragma unroll
+                for (int nn = 0; nn < D / 8; ++nn) {
+                    rb[2 + nn * 8 + 2 * q4] = o[nn][2];
+                    rb[3 + nn * 8 + 2 * q4] = o[nn][3];
+                }
             }
             named_bar_sync(1, kCWarps * 32);
             const int rows = min(p.r, NMT * 16);
@@ -452,11 +465,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const int mtr = hl >> 4, rr = hl & 15;
                 float M = -INFINITY;
 #pragma unroll
-                for (int k = 0; k < NSL; ++k) M = fmaxf(M, red[((k * NMT + mtr) * 16 + rr) * ROWF]);
+                for (int k = 0; k < NSL; ++k) M = fmaxf(M, red[((k * NMT + mtr) * RR + rr) * ROWF]);
                 float acc = 0.f, L = 0.f;
 #pragma unroll
                 for (int k = 0; k < NSL; ++k) {
-                    const float *row = red + ((k * NMT + mtr) * 16 + rr) * ROWF;
+                    const float *row = red + ((k * NMT + mtr) * RR + rr) * ROWF;
                     const float w = fast_exp2(row[0] - M);
                     acc += w * row[2 + col];
                     L += w * row[1];
@@ -663,17 +676,22 @@ cudaError_t set_smem_once(Kern kern, size_t smem) {
     return e;
 }
 
-template <int D, int NMT>
+template <int D, int NMT, int STAGES, int RR>
 struct Bf16Tag {};
 template <int D>
 struct F32Tag {};
 
 int bf16_nmt(int r) { return r <= 16 ? 1 : (r <= 32 ? 2 : 4); }
 
-size_t smem_bf16(int D, int nmt, int B) {
+// Ring depth and reduction rows for a group of r query heads: groups of at
+// most 4 heads use 4-row reduction buffers.
+int bf16_stages(int r) { (void)r; return kStages; }
+int bf16_red_rows(int r) { return r <= 4 ? 4 : 16; }
+
+size_t smem_bf16(int D, int nmt, int B, int stages, int rr) {
     const int nsl = kCWarps / nmt;
-    const size_t red = nsl > 1 ? (size_t)nsl * nmt * 16 * (D + 2) * 4 : 0;
-    return 1024 + (size_t)kStages * 2 * kTile * D * 2 + red + 2 * kStages * 8 + 4 +
+    const size_t red = nsl > 1 ? (size_t)nsl * nmt * rr * (D + 2) * 4 : 0;
+    return 1024 + (size_t)stages * 2 * kTile * D * 2 + red + 2 * (size_t)stages * 8 + 4 +
            (size_t)(B + 1) * 4 + 32 * 4;
 }
 
@@ -682,12 +700,12 @@ size_t smem_f32(int D, int r, int B) {
            (size_t)(B + 1) * 4 + 32 * 4;
 }
 
-template <int D, int NMT>
+template <int D, int NMT, int STAGES, int RR>
 cudaError_t run_bf16(const DecodeParams &p, const CUtensorMap *tmk, const CUtensorMap *tmv,
                      int ctas, cudaStream_t st) {
-    const size_t smem = smem_bf16(D, NMT, p.B);
-    auto kern = decode_split_bf16<D, NMT>;
-    cudaError_t e = set_smem_once<Bf16Tag<D, NMT>>(kern, smem);
+    const size_t smem = smem_bf16(D, NMT, p.B, STAGES, RR);
+    auto kern = decode_split_bf16<D, NMT, STAGES, RR>;
+    cudaError_t e = set_smem_once<Bf16Tag<D, NMT, STAGES, RR>>(kern, smem);
     if (e != cudaSuccess) return e;
     kern<<<ctas, kThreads, smem, st>>>(*tmk, *tmv, p);
     return cudaGetLastError();
@@ -741,7 +759,8 @@ DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, i
 
 size_t decode_smem_bytes(int B, int H, int G, int d_h, int dtype) {
     const int r = H / G;
-    return dtype == GQA_BF16 ? smem_bf16(d_h, bf16_nmt(r), B) : smem_f32(d_h, r, B);
+    return dtype == GQA_BF16 ? smem_bf16(d_h, bf16_nmt(r), B, bf16_stages(r), bf16_red_rows(r))
+                             : smem_f32(d_h, r, B);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUtensorMap *tmv,
@@ -770,13 +789,15 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUt
     if (a.dtype == GQA_BF16) {
         const int nmt = bf16_nmt(p.r);
         if (a.d_h == 128)
-            e = nmt == 1 ? run_bf16<128, 1>(p, tmk, tmv, L.ctas, st)
-              : nmt == 2 ? run_bf16<128, 2>(p, tmk, tmv, L.ctas, st)
-                         : run_bf16<128, 4>(p, tmk, tmv, L.ctas, st);
+            e = p.r <= 4  ? run_bf16<128, 1, kStages, 4>(p, tmk, tmv, L.ctas, st)
+              : nmt == 1  ? run_bf16<128, 1, kStages, 16>(p, tmk, tmv, L.ctas, st)
+              : nmt == 2  ? run_bf16<128, 2, kStages, 16>(p, tmk, tmv, L.ctas, st)
+                          : run_bf16<128, 4, kStages, 16>(p, tmk, tmv, L.ctas, st);
         else
-            e = nmt == 1 ? run_bf16<64, 1>(p, tmk, tmv, L.ctas, st)
-              : nmt == 2 ? run_bf16<64, 2>(p, tmk, tmv, L.ctas, st)
-                         : run_bf16<64, 4>(p, tmk, tmv, L.ctas, st);
+            e = p.r <= 4  ? run_bf16<64, 1, kStages, 4>(p, tmk, tmv, L.ctas, st)
+              : nmt == 1  ? run_bf16<64, 1, kStages, 16>(p, tmk, tmv, L.ctas, st)
+              : nmt == 2  ? run_bf16<64, 2, kStages, 16>(p, tmk, tmv, L.ctas, st)
+                          : run_bf16<64, 4, kStages, 16>(p, tmk, tmv, L.ctas, st);
         if (e != cudaSuccess) return e;
         return a.d_h == 128 ? run_combine<128, true>(p, L.ctas, st) : run_combine<64, true>(p, L.ctas, st);
     }
