@@ -18,6 +18,8 @@
 //      segment).
 //   2. decode_combine: for each (b, i) merges the records of its segment:
 //      M = max m_c, L = sum 2^(m_c - M) l_c, out = sum 2^(m_c - M) o_c / L.
+//   Groups of 16 or more query heads take the tcgen05 split kernel of
+//   decode_tc.cu instead of decode_split_bf16; both write the same records.
 //   Softmax runs in the base-2 domain on scores pre-multiplied by
 //   scale*log2(e), which leaves the result unchanged.
 //
@@ -30,6 +32,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "decode_common.cuh"
 #include "gqa.h"
 #include "internal.h"
 
@@ -37,117 +40,23 @@ namespace gqa {
 
 namespace {
 
-constexpr int kTile = 64;       // tokens per K/V tile, bf16 path
 constexpr int kTileF32 = 32;    // tokens per tile, fp32 path
 constexpr int kStages = 2;      // TMA ring depth per CTA
 constexpr int kCtasPerSm = 2;   // resident split CTAs per SM (2 x 2 stages in flight)
 constexpr int kCWarps = 4;      // consumer warps
 constexpr int kThreads = (kCWarps + 1) * 32;
-constexpr int kHalfBytes = kTile * 128;  // one [64 tokens x 64 dims] bf16 box
 constexpr int kThreadsF32 = 128;
-constexpr int kSplitPMaxLen = 256;  // sequences this short carry P as two bf16 terms
 
-struct DecodeParams {
-    const void *q;
-    const int32_t *seqlens;
-    void *out;
-    int *ws_cu;     // [B+1] tile prefix, written by CTA 0 of the split kernel
-    float2 *ws_ml;  // [n_rec * r]: (max in log2 units, sum)
-    float *ws_o;    // [n_rec * r * d_h]: unnormalised outputs
-    const float *k32, *v32;  // fp32 path only
-    unsigned *status;
-    float scale_log2;
-    int B, H, G, r, T_cap;
-    unsigned long long timeout_ns;
-    int window;  // > 0: attend over the last `window` cached positions only
-};
-
-__device__ __forceinline__ int clamp_len(int T, int T_cap) {
-    return T < 0 ? 0 : (T > T_cap ? T_cap : T);
-}
-
-// Cached positions a sequence attends over: all T_b of them, or with a sliding
-// window of W > 0 only the last min(T_b, W), i.e. [T_b - len, T_b).
-__device__ __forceinline__ int attended_len(int T, const DecodeParams &p) {
-    const int t = clamp_len(T, p.T_cap);
-    return (p.window > 0 && t > p.window) ? p.window : t;
-}
-
-// cu[b] = G * sum_{b' < b} ceil(T_b' / TILE), T clamped to [0, T_cap];
-// cu[B] = total tiles W.  Every thread of the block must call it; blockDim.x
-// is a multiple of 32 and scratch holds 32 ints.
-template <int TILE>
-__device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, bool report) {
-    const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int chunk = (p.B + nt - 1) / nt;
-    const int b0 = min(p.B, tid * chunk), b1 = min(p.B, b0 + chunk);
-    int local = 0;
-    bool bad = false;
-    for (int b = b0; b < b1; ++b) {
-        const int T = p.seqlens[b];
-        bad |= (T < 0 || T > p.T_cap);
-        local += (attended_len(T, p) + TILE - 1) / TILE;
-    }
-    if (bad && report) set_status(p.status, STATUS_SEQLEN);
-    // exclusive block scan of `local`: warp scans, then a scan of the warp totals
-    int incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-    }
-    if (lane == 31) scratch[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        const int nw = nt >> 5;
-        int w = lane < nw ? scratch[lane] : 0;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, w, off);
-            if (lane >= off) w += v;
-        }
-        if (lane < nw) scratch[lane] = w;  // inclusive prefix of warp totals
-        if (lane == nw - 1) cu[p.B] = w * p.G;
-    }
-    __syncthreads();
-    int run = incl - local + (wid > 0 ? scratch[wid - 1] : 0);
-    for (int b = b0; b < b1; ++b) {
-        cu[b] = run * p.G;
-        run += (attended_len(p.seqlens[b], p) + TILE - 1) / TILE;
-    }
-    __syncthreads();
-    return cu[p.B];
-}
-
-// Position in the tile line: sequence b, KV head g, tile j of the segment,
-// tiles per segment of b.
-struct Cursor {
-    int b, g, j, ntb;
-};
-
-__device__ __forceinline__ void cursor_seek(const int *cu, int B, int G, int u, Cursor &c) {
-    int lo = 0, hi = B - 1;  // largest b with cu[b] <= u (then cu[b] <= u < cu[b+1])
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (cu[mid] <= u) lo = mid; else hi = mid - 1;
-    }
-    c.b = lo;
-    c.ntb = (cu[lo + 1] - cu[lo]) / G;
-    const int off = u - cu[lo];
-    c.g = off / c.ntb;
-    c.j = off - c.g * c.ntb;
-}
-
-__device__ __forceinline__ void cursor_next(const int *cu, int B, int G, Cursor &c) {
-    if (++c.j < c.ntb) return;
-    c.j = 0;
-    if (++c.g < G) return;
-    c.g = 0;
-    do {
-        ++c.b;
-    } while (c.b < B && cu[c.b + 1] == cu[c.b]);
-    if (c.b < B) c.ntb = (cu[c.b + 1] - cu[c.b]) / G;
-}
+using dec::attended_len;
+using dec::build_tile_prefix;
+using dec::clamp_len;
+using dec::Cursor;
+using dec::cursor_next;
+using dec::cursor_seek;
+using dec::DecodeParams;
+using dec::kHalfBytes;
+using dec::kSplitPMaxLen;
+using dec::kTile;
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -415,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         la += __shfl_xor_sync(0xffffffffu, la, 2);
         lb += __shfl_xor_sync(0xffffffffu, lb, 1);
         lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-        const long long rec = (long long)blockIdx.x + bg;
+        const long long rec = (long long)blockIdx.x + bg;  // rpp = 1
         if (NSL == 1) {
             const int hl_a = mt * 16 + g8, hl_b = hl_a + 8;
             if (!dead && hl_a < p.r) {
@@ -575,7 +484,7 @@ __global__ void __launch_bounds__(kThreadsF32)
         cursor_next(cu, p.B, p.G, c);
         const bool piece_end = (u + 1 == u_end) || (c.b * p.G + c.g != bg);
         if (piece_end) {
-            const long long rec = (long long)blockIdx.x + bg;
+            const long long rec = (long long)blockIdx.x + bg;  // rpp = 1
             for (int i = tid; i < p.r * D; i += blockDim.x) p.ws_o[rec * p.r * D + i] = st_o[i];
             for (int i = tid; i < p.r; i += blockDim.x)
                 p.ws_ml[rec * p.r + i] = make_float2(st_m[i], st_l[i]);
@@ -586,19 +495,30 @@ __global__ void __launch_bounds__(kThreadsF32)
 
 // ----------------------------------------------------------------- combine
 
-template <int D, bool BF16_OUT>
-__global__ void __launch_bounds__(128) decode_combine(const DecodeParams p, int C) {
+// One CTA of NW warps per output row (b, i).  Warp w merges records w,
+// w + NW, ... of the row's segment (record index i = piece * RPP + slice),
+// issuing the loads of up to kCombBatch records at once and keeping a running
+// (max, sum, o); the warps' results are then merged in a fixed order
+// (deterministic results).  A record with m = -inf (a slice that saw no
+// position) adds nothing.  NW is 16, 8 or 4 (see run_combine).
+constexpr int kCombBatch = 8;
+
+template <int D, bool BF16_OUT, int RPP, int NW>
+__global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, int C) {
+    constexpr int kCombWarps = NW;
     pdl_wait_primary();  // the split kernel's records are complete and visible
+    constexpr int PER = D / 32;
+    __shared__ float red_m[kCombWarps], red_l[kCombWarps];
+    __shared__ __align__(16) float red_o[kCombWarps][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long row = (long long)blockIdx.x * 4 + warp;  // b*H + h
-    if (row >= (long long)p.B * p.H) return;
+    const long long row = blockIdx.x;  // b*H + h
     const int b = (int)(row / p.H), h = (int)(row % p.H);
     const int g = h / p.r, hl = h - g * p.r;
     const int bg = b * p.G + g;
-    constexpr int PER = D / 32;
     float acc[PER];
 #pragma unroll
     for (int k = 0; k < PER; ++k) acc[k] = 0.f;
+    float M = -INFINITY, L = 0.f;
     const int *cu = p.ws_cu;
     const int ntb = (cu[b + 1] - cu[b]) / p.G;
     if (ntb > 0) {
@@ -606,39 +526,73 @@ __global__ void __launch_bounds__(128) decode_combine(const DecodeParams p, int 
         const long long s0 = cu[b] + (long long)g * ntb, s1 = s0 + ntb;
         const int c_lo = (int)(((s0 + 1) * C - 1) / W);
         const int c_hi = (int)((s1 * C - 1) / W);
-        // CTAs whose share is empty (more CTAs than tiles) wrote no record.
-        // One pass: running maximum, with the partial sums rescaled as it grows.
-        auto empty_share = [&](int c) { return (long long)c * W / C == (long long)(c + 1) * W / C; };
-        float M = -INFINITY, L = 0.f;
-#pragma unroll 4
-        for (int c = c_lo; c <= c_hi; ++c) {
-            if (empty_share(c)) continue;
-            const long long rec = (long long)c + bg;
-            const float2 ml = p.ws_ml[rec * p.r + hl];
-            const float *src = p.ws_o + (rec * p.r + hl) * D + lane * PER;
-            float v[PER];
-            if constexpr (PER == 4) {
-                const float4 t = *reinterpret_cast<const float4 *>(src);
-                v[0] = t.x;
-                v[1] = t.y;
-                v[2] = t.z;
-                v[3] = t.w;
-            } else {
-                const float2 t = *reinterpret_cast<const float2 *>(src);
-                v[0] = t.x;
-                v[1] = t.y;
+        const int n = (c_hi - c_lo + 1) * RPP;
+        // With fewer tiles than CTAs some shares are empty; those CTAs wrote no record.
+        const bool may_skip = W < C;
+        for (int i0 = warp; i0 < n; i0 += kCombWarps * kCombBatch) {
+            float2 ml[kCombBatch];
+            float v[kCombBatch][PER];
+#pragma unroll
+            for (int j = 0; j < kCombBatch; ++j) {
+                const int i = i0 + j * kCombWarps;
+                const int c = c_lo + i / RPP;
+                ml[j] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                for (int k = 0; k < PER; ++k) v[j][k] = 0.f;
+                if (i >= n || (may_skip && (long long)c * W / C == (long long)(c + 1) * W / C)) continue;
+                const long long rec = ((long long)c + bg) * RPP + i % RPP;
+                ml[j] = p.ws_ml[rec * p.r + hl];
+                const float *src = p.ws_o + (rec * p.r + hl) * D + lane * PER;
+                if constexpr (PER == 4) {
+                    const float4 t = *reinterpret_cast<const float4 *>(src);
+                    v[j][0] = t.x;
+                    v[j][1] = t.y;
+                    v[j][2] = t.z;
+                    v[j][3] = t.w;
+                } else {
+                    const float2 t = *reinterpret_cast<const float2 *>(src);
+                    v[j][0] = t.x;
+                    v[j][1] = t.y;
+                }
             }
-            const float Mn = fmaxf(M, ml.x);
-            const float a = fast_exp2(M - Mn), w = fast_exp2(ml.x - Mn);
-            L = L * a + w * ml.y;
 #pragma unroll
-            for (int k = 0; k < PER; ++k) acc[k] = acc[k] * a + w * v[k];
-            M = Mn;
+            for (int j = 0; j < kCombBatch; ++j) {
+                const float Mn = fmaxf(M, ml[j].x);
+                if (Mn == -INFINITY) continue;  // nothing seen yet
+                const float a = fast_exp2(M - Mn), w = fast_exp2(ml[j].x - Mn);
+                L = L * a + w * ml[j].y;
+#pragma unroll
+                for (int k = 0; k < PER; ++k) acc[k] = acc[k] * a + w * v[j][k];
+                M = Mn;
+            }
         }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-        for (int k = 0; k < PER; ++k) acc[k] *= inv;
     }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) red_o[warp][lane * PER + k] = acc[k];
+    if (lane == 0) {
+        red_m[warp] = M;
+        red_l[warp] = L;
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    float Mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) Mt = fmaxf(Mt, red_m[w]);
+    float Lt = 0.f;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc[k] = 0.f;
+    if (Mt != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kCombWarps; ++w) {
+            const float f = fast_exp2(red_m[w] - Mt);  // 0 for a warp that merged nothing
+            Lt = fmaf(f, red_l[w], Lt);
+#pragma unroll
+            for (int k = 0; k < PER; ++k) acc[k] = fmaf(f, red_o[w][lane * PER + k], acc[k]);
+        }
+    }
+    const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc[k] *= inv;
     if constexpr (BF16_OUT) {
         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + row * D + lane * PER;
         if constexpr (PER == 4)
@@ -721,11 +675,11 @@ cudaError_t run_f32(const DecodeParams &p, int ctas, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <int D, bool BF16_OUT>
-cudaError_t run_combine(const DecodeParams &p, int ctas, cudaStream_t st) {
+template <int D, bool BF16_OUT, int NW>
+cudaError_t run_combine_nw(const DecodeParams &p, int ctas, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(((long long)p.B * p.H + 3) / 4));
-    cfg.blockDim = dim3(128);
+    cfg.gridDim = dim3((unsigned)((long long)p.B * p.H));
+    cfg.blockDim = dim3(NW * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -733,7 +687,24 @@ cudaError_t run_combine(const DecodeParams &p, int ctas, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT>, p, ctas);
+    switch (p.rpp) {
+        case 1: return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT, 1, NW>, p, ctas);
+        case 2: return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT, 2, NW>, p, ctas);
+        case 4: return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT, 4, NW>, p, ctas);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int D, bool BF16_OUT>
+cudaError_t run_combine(const DecodeParams &p, int ctas, cudaStream_t st) {
+    // Records of one row: about (CTAs per segment + 1) pieces of rpp records.
+    // Wide CTAs (16 warps, one per SM by registers) only when the rows are few
+    // enough to fit one wave and have records for the extra warps.
+    const long long segs = (long long)p.B * p.G, rows = (long long)p.B * p.H;
+    const long long recs = (((long long)ctas + segs - 1) / segs + 1) * p.rpp;
+    if (rows <= 148 && recs > 16) return run_combine_nw<D, BF16_OUT, 16>(p, ctas, st);
+    if (rows <= 3 * 148 && recs > 8) return run_combine_nw<D, BF16_OUT, 8>(p, ctas, st);
+    return run_combine_nw<D, BF16_OUT, 4>(p, ctas, st);
 }
 
 }  // namespace
@@ -744,12 +715,14 @@ DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, i
     const int r = H / G;
     const int tile = dtype == GQA_BF16 ? kTile : kTileF32;
     const long long max_tiles = (long long)B * G * ((T_cap + tile - 1) / tile);
+    const bool tc = dtype == GQA_BF16 && dec::tc_eligible(r, d_h, B);
     long long ctas = force_ctas > 0 ? force_ctas
-                                    : (long long)num_sms * (dtype == GQA_BF16 ? kCtasPerSm : 1);
+                                    : (long long)num_sms * (dtype == GQA_BF16 && !tc ? kCtasPerSm : 1);
     if (ctas > max_tiles) ctas = max_tiles;
     if (ctas < 1) ctas = 1;
     L.ctas = (int)ctas;
-    L.n_rec = ctas + (long long)B * G;
+    L.rpp = tc ? dec::tc_records_per_piece(r) : 1;
+    L.n_rec = L.rpp * (ctas + (long long)B * G);
     L.off_cu = 0;
     L.off_ml = align256((size_t)(B + 1) * 4);
     L.off_o = L.off_ml + align256((size_t)L.n_rec * r * sizeof(float2));
@@ -759,6 +732,7 @@ DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, i
 
 size_t decode_smem_bytes(int B, int H, int G, int d_h, int dtype) {
     const int r = H / G;
+    if (dtype == GQA_BF16 && dec::tc_eligible(r, d_h, B)) return dec::tc_smem_bytes(d_h, B);
     return dtype == GQA_BF16 ? smem_bf16(d_h, bf16_nmt(r), B, bf16_stages(r), bf16_red_rows(r))
                              : smem_f32(d_h, r, B);
 }
@@ -785,10 +759,13 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUt
     p.T_cap = a.T_cap;
     p.timeout_ns = a.timeout_ns;
     p.window = a.window;
+    p.rpp = L.rpp;
     cudaError_t e;
     if (a.dtype == GQA_BF16) {
         const int nmt = bf16_nmt(p.r);
-        if (a.d_h == 128)
+        if (dec::tc_eligible(p.r, a.d_h, a.B)) {
+            e = dec::run_split_tc(p, tmk, tmv, a.d_h, L.ctas, st);
+        } else if (a.d_h == 128)
             e = p.r <= 4  ? run_bf16<128, 1, kStages, 4>(p, tmk, tmv, L.ctas, st)
               : nmt == 1  ? run_bf16<128, 1, kStages, 16>(p, tmk, tmv, L.ctas, st)
               : nmt == 2  ? run_bf16<128, 2, kStages, 16>(p, tmk, tmv, L.ctas, st)

@@ -1,0 +1,142 @@
+// decode_common.cuh -- the split-KV partition shared by the decode kernels.
+//
+// The cache tiles of all (b, g) segments ("Grouped-Query Attention",
+// llm-arch-kb, section 1: G key/value heads per sequence) are laid end to end
+// and cut into gridDim.x equal shares.  CTA c takes share c; a share may cover
+// the tail of one segment and the head of the next.  For each piece (the part
+// of one segment inside one share) the CTA emits rpp partial records
+// (running max m in log2 units, sum l, unnormalised o[d_h]) per query head at
+// record indices rpp*(c + segment) + [0, rpp): distinct for all pieces, since
+// two pieces with equal c + segment would need an earlier CTA to hold a later
+// segment.  A record whose slice saw no position has m = -inf, l = 0, o = 0.
+#pragma once
+
+#include "common.cuh"
+
+namespace gqa {
+namespace dec {
+
+constexpr int kTile = 64;                // tokens per K/V tile, bf16 kernels
+constexpr int kHalfBytes = kTile * 128;  // one [64 tokens x 64 dims] bf16 box
+constexpr int kSplitPMaxLen = 256;       // sequences this short carry P as two bf16 terms
+
+struct DecodeParams {
+    const void *q;
+    const int32_t *seqlens;
+    void *out;
+    int *ws_cu;     // [B+1] tile prefix, written by CTA 0 of the split kernel
+    float2 *ws_ml;  // [n_rec * r]: (max in log2 units, sum)
+    float *ws_o;    // [n_rec * r * d_h]: unnormalised outputs
+    const float *k32, *v32;  // fp32 path only
+    unsigned *status;
+    float scale_log2;
+    int B, H, G, r, T_cap;
+    unsigned long long timeout_ns;
+    int window;  // > 0: attend over the last `window` cached positions only
+    int rpp;     // records per piece: piece (c, segment) owns records rpp*(c+segment) + [0, rpp)
+};
+
+__device__ __forceinline__ int clamp_len(int T, int T_cap) {
+    return T < 0 ? 0 : (T > T_cap ? T_cap : T);
+}
+
+// Cached positions a sequence attends over: all T_b of them, or with a sliding
+// window of W > 0 only the last min(T_b, W), i.e. [T_b - len, T_b).
+__device__ __forceinline__ int attended_len(int T, const DecodeParams &p) {
+    const int t = clamp_len(T, p.T_cap);
+    return (p.window > 0 && t > p.window) ? p.window : t;
+}
+
+// cu[b] = G * sum_{b' < b} ceil(len_b' / TILE), len as attended_len;
+// cu[B] = total tiles.  Every thread of the block must call it; blockDim.x
+// is a multiple of 32 and scratch holds 32 ints.  When tb is given it
+// receives T_b clamped to [0, T_cap] for every b.
+template <int TILE>
+__device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, bool report, int *tb = nullptr) {
+    const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int chunk = (p.B + nt - 1) / nt;
+    const int b0 = min(p.B, tid * chunk), b1 = min(p.B, b0 + chunk);
+    int local = 0;
+    bool bad = false;
+    for (int b = b0; b < b1; ++b) {
+        const int T = p.seqlens[b];
+        bad |= (T < 0 || T > p.T_cap);
+        local += (attended_len(T, p) + TILE - 1) / TILE;
+        if (tb) tb[b] = clamp_len(T, p.T_cap);
+    }
+    if (bad && report) set_status(p.status, STATUS_SEQLEN);
+    // exclusive block scan of `local`: warp scans, then a scan of the warp totals
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) scratch[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        const int nw = nt >> 5;
+        int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += v;
+        }
+        if (lane < nw) scratch[lane] = w;  // inclusive prefix of warp totals
+        if (lane == nw - 1) cu[p.B] = w * p.G;
+    }
+    __syncthreads();
+    int run = incl - local + (wid > 0 ? scratch[wid - 1] : 0);
+    for (int b = b0; b < b1; ++b) {
+        cu[b] = run * p.G;
+        run += (attended_len(p.seqlens[b], p) + TILE - 1) / TILE;
+    }
+    __syncthreads();
+    return cu[p.B];
+}
+
+// Position in the tile line: sequence b, KV head g, tile j of the segment,
+// tiles per segment of b.
+struct Cursor {
+    int b, g, j, ntb;
+};
+
+__device__ __forceinline__ void cursor_seek(const int *cu, int B, int G, int u, Cursor &c) {
+    int lo = 0, hi = B - 1;  // largest b with cu[b] <= u (then cu[b] <= u < cu[b+1])
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cu[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    c.b = lo;
+    c.ntb = (cu[lo + 1] - cu[lo]) / G;
+    const int off = u - cu[lo];
+    c.g = off / c.ntb;
+    c.j = off - c.g * c.ntb;
+}
+
+__device__ __forceinline__ void cursor_next(const int *cu, int B, int G, Cursor &c) {
+    if (++c.j < c.ntb) return;
+    c.j = 0;
+    if (++c.g < G) return;
+    c.g = 0;
+    do {
+        ++c.b;
+    } while (c.b < B && cu[c.b + 1] == cu[c.b]);
+    if (c.b < B) c.ntb = (cu[c.b + 1] - cu[c.b]) / G;
+}
+
+// ------------------------------------------------- tensor-core split kernel
+
+// Groups of at least this many query heads use the tcgen05 split kernel.
+constexpr int kTcMinHeads = 16;
+
+bool tc_eligible(int r, int d_h, int B);
+size_t tc_smem_bytes(int d_h, int B);
+// Records the tcgen05 kernel writes per piece (one per token slice).
+int tc_records_per_piece(int r);
+// Launches the tcgen05 split kernel on `ctas` CTAs (one per SM).
+cudaError_t run_split_tc(const DecodeParams &p, const CUtensorMap *tmk, const CUtensorMap *tmv, int d_h, int ctas,
+                         cudaStream_t st);
+
+}  // namespace dec
+}  // namespace gqa

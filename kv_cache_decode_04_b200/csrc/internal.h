@@ -32,13 +32,16 @@ struct DecodeArgs {
 // Workspace layout, all offsets 256-byte aligned.
 struct DecodeLayout {
     int ctas;          // split CTAs of the first kernel
-    long long n_rec;   // partial records: ctas + B*G
+    int rpp;           // partial records per piece
+    long long n_rec;   // partial records: rpp * (ctas + B*G)
     size_t off_cu, off_ml, off_o, total;
 };
 
 DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, int num_sms,
                            int force_ctas);
 size_t decode_smem_bytes(int B, int H, int G, int d_h, int dtype);
+// Split kernel + combine.  tmk/tmv ([B*G*T_cap, d_h], boxes of [64 x 64])
+// for every bf16 call.
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUtensorMap *tmv,
                           cudaStream_t stream);
 
