@@ -677,6 +677,22 @@ cudaError_t run_f32(const DecodeParams &p, int ctas, cudaStream_t st) {
 
 template <int D, bool BF16_OUT, int NW>
 cudaError_t run_combine_nw(const DecodeParams &p, int ctas, cudaStream_t st) {
+    // The split kernels before it run with (nearly) all of an SM's shared
+    // memory; asking for the same carveout here spares every call an L1/shared
+    // memory reconfiguration of the SMs between the two kernels.
+    static int carveout_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (carveout_dev != dev) {
+        const int pct = (int)cudaSharedmemCarveoutMaxShared;
+        for (auto kern : {decode_combine<D, BF16_OUT, 1, NW>, decode_combine<D, BF16_OUT, 2, NW>,
+                          decode_combine<D, BF16_OUT, 4, NW>}) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
+            if (e != cudaSuccess) return e;
+        }
+        carveout_dev = dev;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((long long)p.B * p.H));
     cfg.blockDim = dim3(NW * 32);

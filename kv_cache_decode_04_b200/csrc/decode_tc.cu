@@ -22,9 +22,9 @@
 // outside the slice, so the P.V of copy k accumulates the slice's share of the
 // output.  The copies cost no tensor time (the instruction is M = 128 either
 // way) and spread the softmax over all four SM sub-partitions.  Each slice
-// keeps its own online softmax and writes its own partial record per piece
-// (records per piece = NREP); decode_combine merges them with the other
-// pieces' records.
+// keeps its own online softmax; at the end of a piece the slices' partial
+// results are merged in shared memory into the piece's one record, which
+// decode_combine merges with the other pieces' records.
 //
 // Partition and records follow decode_common.cuh, with 128-position tiles.
 //
@@ -77,9 +77,10 @@ struct TcLayout {
     static constexpr int OFF_RING = 0;
     static constexpr int OFF_BAR = OFF_RING + STAGES * STAGE_BYTES;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int OFF_XP = OFF_BAR + BAR_BYTES;    // record transpose, [4 warps][32][33] floats
+    static constexpr int OFF_XP = OFF_BAR + BAR_BYTES;    // record merge, [4 warps][32][33] floats
     static constexpr int XP_BYTES = 4 * 32 * 33 * 4;
-    static constexpr int OFF_CU = OFF_XP + XP_BYTES;      // cu[B+1], scratch[32], tb[B]
+    static constexpr int OFF_ML = OFF_XP + XP_BYTES;      // slices' (m, l), [4 warps][32] float2
+    static constexpr int OFF_CU = OFF_ML + 4 * 32 * 8;    // cu[B+1], scratch[32], tb[B]
 };
 
 template <int D>
@@ -159,7 +160,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *p_ready = s_full + kNS;        // [kNS] P of the tile in S buffer i
     uint64_t *pv_done = p_ready + kNS;       // [kNS] P.V of the tile in S buffer i
     uint64_t *drain = pv_done + kNS;         // [2] one per MMA-issuing thread
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 2);
+    uint64_t *ep_bar = drain + 2;            // the softmax warps' record merge (128 arrivals a phase)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ep_bar + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     int *cu = reinterpret_cast<int *>(sm + Lay::OFF_CU);
     int *scratch = cu + p.B + 1;
@@ -182,6 +184,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&p_ready[s], 128);
             mbar_init(&pv_done[s], 1);
         }
+        mbar_init(ep_bar, 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -367,6 +370,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         int piece = -1;
+        uint32_t ep_phase = 0;
+        // all 128 softmax threads meet (bounded: false when a wait ran out)
+        auto ep_sync = [&]() {
+            mbar_arrive(ep_bar);
+            const bool done = warp_wait(ep_bar, ep_phase & 1, p.timeout_ns);
+            ++ep_phase;
+            return done;
+        };
         if (u_begin < u_end) {  // the first piece's rows
             Cursor c0;
             cursor_seek(cu, p.B, p.G, u_begin, c0);
@@ -496,32 +507,62 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
             if (t.last) {
-                // piece done: wait for its last P.V, then write this slice's record
+                // Piece done: wait for its last P.V, then merge the NREP slices' partial
+                // results of every head into the piece's record:
+                //   M = max_k m_k, L = sum_k 2^(m_k - M) l_k, o = sum_k 2^(m_k - M) O_k.
+                // The warps of one head block (same warp % NSW) exchange (m, l) and their
+                // scaled O rows through shared memory, 32 columns at a time; each warp
+                // then adds up every NREP-th row in slice order and writes it with
+                // coalesced 128-byte stores.
                 if (!warp_wait(&pv_done[sb], (it / kNS) & 1, p.timeout_ns)) {
                     ok = false;
                     return false;
                 }
                 tc::fence_after();
-                const long long rec = ((long long)blockIdx.x + t.bg) * NREP + k;
-                // rows head0..head0+31 of the record are consecutive [d_h] float rows:
-                // each 32-column chunk goes through a [32][33] transpose so that one
-                // store writes 32 consecutive floats of one row
-                const int head0 = (warp % NSW) * 32;
-                float *xp = reinterpret_cast<float *>(sm + Lay::OFF_XP) + warp * 32 * 33;
-                float *dst0 = p.ws_o + (rec * p.r + head0) * D;
-                const int nrows = min(32, p.r - head0);
+                float2 *mlx = reinterpret_cast<float2 *>(sm + Lay::OFF_ML);
+                float *xp = reinterpret_cast<float *>(sm + Lay::OFF_XP);
+                const int hb = warp % NSW;
+                mlx[warp * 32 + lane] = make_float2(m, l);
+                if (!ep_sync()) {
+                    ok = false;
+                    return false;
+                }
+                float M = -INFINITY;
+#pragma unroll
+                for (int kk = 0; kk < NREP; ++kk) M = fmaxf(M, mlx[(kk * NSW + hb) * 32 + lane].x);
+                float L = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < NREP; ++kk) {
+                    const float2 v = mlx[(kk * NSW + hb) * 32 + lane];
+                    L += v.x == -INFINITY ? 0.f : fast_exp2(v.x - M) * v.y;
+                }
+                const float wgt = m == -INFINITY ? 0.f : fast_exp2(m - M);
+                const long long rec = (long long)blockIdx.x + t.bg;
+                float *dst0 = p.ws_o + (rec * p.r + hb * 32) * D;
+                const int nrows = min(32, p.r - hb * 32);
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t orow[32];
                     tc::ld32(tO + c * 32, orow);
                     tc::wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = __uint_as_float(orow[e]);
-                    __syncwarp();
-                    for (int i = 0; i < nrows; ++i) dst0[(size_t)i * D + c * 32 + lane] = xp[i * 33 + lane];
-                    __syncwarp();
+                    for (int e = 0; e < 32; ++e) xp[(warp * 32 + lane) * 33 + e] = __uint_as_float(orow[e]) * wgt;
+                    if (!ep_sync()) {
+                        ok = false;
+                        return false;
+                    }
+                    for (int i = k; i < nrows; i += NREP) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int kk = 0; kk < NREP; ++kk) acc += xp[((kk * NSW + hb) * 32 + i) * 33 + lane];
+                        dst0[(size_t)i * D + c * 32 + lane] = acc;
+                    }
+                    if (!ep_sync()) {
+                        ok = false;
+                        return false;
+                    }
                 }
-                if (valid) p.ws_ml[rec * p.r + head] = make_float2(m, l);
+                if (k == 0 && valid) p.ws_ml[rec * p.r + head] = make_float2(M, L);
             }
             return true;
         });
@@ -563,7 +604,10 @@ bool tc_eligible(int r, int d_h, int B) {
 
 size_t tc_smem_bytes(int d_h, int B) { return d_h == 128 ? smem_tc<128>(B) : smem_tc<64>(B); }
 
-int tc_records_per_piece(int r) { return r > 32 ? 2 : 4; }
+int tc_records_per_piece(int r) {
+    (void)r;
+    return 1;  // the slices of a piece are merged in the split kernel
+}
 
 cudaError_t run_split_tc(const DecodeParams &p, const CUtensorMap *tmk, const CUtensorMap *tmv, int d_h, int ctas,
                          cudaStream_t st) {
