@@ -172,6 +172,7 @@ BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 
 class Decode:
     kind = "decode"
+    graphable = True  # a step is a pure function of the resident inputs
 
     def __init__(self, name, gqa, device="cuda"):
         w = gi.WORKLOADS[name]
@@ -267,6 +268,7 @@ class Decode:
 
 class Prefill:
     kind = "prefill"
+    graphable = True
 
     def __init__(self, name, gqa, device="cuda"):
         w = gi.WORKLOADS[name]
@@ -325,6 +327,7 @@ class Prefill:
 
 class MeanPool:
     kind = "meanpool"
+    graphable = True
 
     def __init__(self, name, gqa, device="cuda"):
         w = gi.WORKLOADS[name]
@@ -456,22 +459,64 @@ def make(name, gqa):
 
 # ------------------------------------------------------------------ timing
 
+GRAPH_CHUNK = 50  # steps per captured CUDA graph
+
+
+def _capture(wl, n):
+    """A CUDA graph of n consecutive steps of wl (the same kernels, arguments
+    and stream order as n eager calls), or None when capture fails."""
+    if n <= 0:
+        return None
+    try:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(n):
+                wl.step()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        return g
+    except Exception:  # noqa: BLE001 -- any capture failure means: launch eagerly
+        torch.cuda.synchronize()
+        return None
+
+
 def time_steps(wl, steps, warmup, world, clocks=None):
     """W untimed steps, then K steps between a barrier + synchronize on both
     sides, timed with CUDA events on the launching stream.  Returns seconds
-    per step (max over ranks)."""
+    per step (max over ranks).  Workloads whose step is a pure function of
+    resident inputs replay it from CUDA graphs of GRAPH_CHUNK steps (exactly
+    K steps in all); wl.launch records which launch mode was timed."""
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         wl.step()
     torch.cuda.synchronize()
+    graphs = None
+    if getattr(wl, "graphable", False):
+        full, rem = divmod(steps, GRAPH_CHUNK)
+        g_full = _capture(wl, GRAPH_CHUNK) if full else None
+        g_rem = _capture(wl, rem) if rem else None
+        if (g_full is not None or not full) and (g_rem is not None or not rem):
+            graphs = (g_full, full, g_rem)
+            g_full and g_full.replay()  # one untimed replay: the graphs' first launch
+            torch.cuda.synchronize()
+    wl.launch = ("cuda_graph, %d steps per graph" % GRAPH_CHUNK) if graphs else "eager"
     barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ctx = clocks if clocks is not None else _Null()
     with ctx:
         ev0.record(stream)
-        for _ in range(steps):
-            wl.step()
+        if graphs:
+            g_full, full, g_rem = graphs
+            for _ in range(full):
+                g_full.replay()
+            if g_rem is not None:
+                g_rem.replay()
+        else:
+            for _ in range(steps):
+                wl.step()
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -607,7 +652,8 @@ def measure_row(name, gqa, peaks, which, world, target_s=0.4):
     sps0 = probe_step_time(wl)
     steps = steps_for(sps0, target_s)
     sps = time_steps(wl, steps, max(3, min(50, steps // 10)), world)
-    row = {"config": wl.config(), "steps": steps, "ms_per_step": sps * 1e3, "dtype": wl.dtype}
+    row = {"config": dict(wl.config(), launch=wl.launch), "steps": steps, "ms_per_step": sps * 1e3,
+           "dtype": wl.dtype}
     row.update(wl.metric(sps, world))
     row["roofline"] = wl.roofline(sps, peaks, which, long_run=sps * steps > 1.0)
     del wl
@@ -659,7 +705,8 @@ def main():
             "steps": args.steps, "warmup": warmup, "ms_per_step": sps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic",
-            "config": dict(wl.config(), parallelism="replicas, one independent batch per rank",
+            "config": dict(wl.config(), launch=wl.launch,
+                           parallelism="replicas, one independent batch per rank",
                            l2="inputs larger than L2 (KV %.0f MB vs 126 MB L2), no flush"
                            % (getattr(wl, "bytes", 0) / 1e6)),
             "roofline": roof, "clocks": dict(csum, remeasured=remeasured),

@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
     }
+    pdl_wait_primary();  // inputs written by the kernels before this one are visible
     const int W = build_tile_prefix<kTile>(p, cu, scratch, blockIdx.x == 0);
     if (blockIdx.x == 0)
         for (int i = tid; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
@@ -411,6 +412,7 @@ __global__ void __launch_bounds__(kThreadsF32)
     int *scratch = cu + p.B + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_wait_primary();  // inputs written by the kernels before this one are visible
     const int W = build_tile_prefix<kTileF32>(p, cu, scratch, blockIdx.x == 0);
     if (blockIdx.x == 0)
         for (int i = tid; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
@@ -507,6 +509,7 @@ template <int D, bool BF16_OUT, int RPP, int NW>
 __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, int C) {
     constexpr int kCombWarps = NW;
     pdl_wait_primary();  // the split kernel's records are complete and visible
+    pdl_launch_dependents();  // the next decode's split kernel may start its prologue
     constexpr int PER = D / 32;
     __shared__ float red_m[kCombWarps], red_l[kCombWarps];
     __shared__ __align__(16) float red_o[kCombWarps][D];
@@ -661,8 +664,7 @@ cudaError_t run_bf16(const DecodeParams &p, const CUtensorMap *tmk, const CUtens
     auto kern = decode_split_bf16<D, NMT, STAGES, RR>;
     cudaError_t e = set_smem_once<Bf16Tag<D, NMT, STAGES, RR>>(kern, smem);
     if (e != cudaSuccess) return e;
-    kern<<<ctas, kThreads, smem, st>>>(*tmk, *tmv, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(ctas), dim3(kThreads), smem, st, *tmk, *tmv, p);
 }
 
 template <int D>
@@ -671,8 +673,7 @@ cudaError_t run_f32(const DecodeParams &p, int ctas, cudaStream_t st) {
     auto kern = decode_split_f32<D>;
     cudaError_t e = set_smem_once<F32Tag<D>>(kern, smem);
     if (e != cudaSuccess) return e;
-    kern<<<ctas, kThreadsF32, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(ctas), dim3(kThreadsF32), smem, st, p);
 }
 
 template <int D, bool BF16_OUT, int NW>

@@ -125,6 +125,25 @@ __device__ __forceinline__ void cursor_next(const int *cu, int B, int G, Cursor 
     if (c.b < B) c.ntb = (cu[c.b + 1] - cu[c.b]) / G;
 }
 
+// Launches a split kernel as a programmatic dependent of the work before it in
+// the stream: its prologue (barrier set-up, TMEM allocation, tensor-map
+// prefetch) may overlap the tail of that work; the kernel calls
+// griddepcontrol.wait before it reads any input.
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // ------------------------------------------------- tensor-core split kernel
 
 // Groups of at least this many query heads use the tcgen05 split kernel.

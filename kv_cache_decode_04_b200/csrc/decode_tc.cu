@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc::tmem_alloc(tmem_slot, kTcTmemCols);
         tc::fence_before();
     }
+    pdl_wait_primary();  // inputs written by the kernels before this one are visible
     const int W = build_tile_prefix<kTT>(p, cu, scratch, blockIdx.x == 0, tb);  // syncs the block
     if (blockIdx.x == 0)
         for (int i = tid; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
@@ -592,8 +593,7 @@ cudaError_t run(const DecodeParams &p, const CUtensorMap *tmk, const CUtensorMap
         if (e != cudaSuccess) return e;
         set_dev = dev;
     }
-    kern<<<ctas, kTcThreads, smem, st>>>(*tmk, *tmv, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(ctas), dim3(kTcThreads), smem, st, *tmk, *tmv, p);
 }
 
 }  // namespace
