@@ -368,16 +368,35 @@ class MeanPool:
                 "sample": "the whole conversion (both W_K and W_V)"}
 
 
+L2_ROTATE_BYTES = 256 << 20  # > 2x the 126 MB L2
+
+
+def rotation(nbytes):
+    """Copies of a weight set needed for the steps' working set to exceed L2."""
+    return max(1, -(-L2_ROTATE_BYTES // max(1, nbytes)))
+
+
 class QkvAppend:
-    """One decode token's Q/K/V projections with the KV-cache append."""
+    """One decode token's Q/K/V projections with the KV-cache append.
+
+    The weights (48 MB for the 7B shape) would fit in L2, so step i reads copy
+    i mod n of them, with n copies spanning more than twice the L2; every step
+    writes the same k/v rows and q, so repeated steps are identical work."""
     kind = "qkv"
+    graphable = True
 
     def __init__(self, name, gqa, device="cuda"):
         w = gi.WORKLOADS[name]
         self.name, self.w, self.gqa = name, w, gqa
         x = gi.qkv_inputs(w["B"], w["d"], w["H"], w["G"], w["d_h"], w["T"], w["dtype"], seed=0)
         self.x = x
-        self.h, self.wq, self.wk, self.wv = (t.to(device) for t in (x.h, x.W_Q, x.W_K, x.W_V))
+        self.h = x.h.to(device)
+        wbytes = sum(t.numel() * t.element_size() for t in (x.W_Q, x.W_K, x.W_V)) + self._extra_weight_bytes()
+        self.n_sets = rotation(wbytes)
+        self.sets = [tuple(t.to(device) for t in (x.W_Q, x.W_K, x.W_V)) for _ in range(self.n_sets)]
+        self.wq, self.wk, self.wv = self.sets[0]
+        self.i = 0
+        self.weight_mb = wbytes / 1e6
         self.kc, self.vc = x.k_cache.to(device), x.v_cache.to(device)
         self.sl = x.seqlens.to(device)
         self.q = torch.empty((x.B, x.H, x.d_h), dtype=x.h.dtype, device=device)
@@ -389,14 +408,25 @@ class QkvAppend:
         self.launches_per_step = (x.B + 31) // 32
         self.dtype = "bf16"
 
+    def _extra_weight_bytes(self):
+        return 0
+
+    def _next_set(self):
+        ws = self.sets[self.i % self.n_sets]
+        self.i += 1
+        return ws
+
     def step(self, stream=None):
-        self.gqa.qkv_append(self.h, self.wq, self.wk, self.wv, self.kc, self.vc, self.sl,
+        wq, wk, wv = self._next_set()
+        self.gqa.qkv_append(self.h, wq, wk, wv, self.kc, self.vc, self.sl,
                             q_out=self.q, seqlens_out=self.sl_out, stream=stream)
 
     def config(self):
         x = self.x
         return {"workload": self.name, "B": x.B, "d": x.d, "H": x.H, "G": x.G, "d_h": x.d_h,
-                "T_cap": x.T_cap}
+                "T_cap": x.T_cap,
+                "l2": "weights rotate over %d copies of %.0f MB (> 126 MB L2), no flush"
+                      % (self.n_sets, self.weight_mb)}
 
     def metric(self, sps, n_ranks):
         return {"value": n_ranks * self.bytes / sps / 1e9, "unit": "GB/s"}
@@ -425,7 +455,9 @@ class LayerDecode(QkvAppend):
         x = self.x
         gen = torch.Generator().manual_seed(1)
         D = x.H * x.d_h
-        self.wo = (torch.randn(D, x.d, generator=gen) * D ** -0.5).to(x.h.dtype).to(device)
+        wo = (torch.randn(D, x.d, generator=gen) * D ** -0.5).to(x.h.dtype)
+        self.wos = [wo.to(device) for _ in range(self.n_sets)]
+        self.wo = self.wos[0]
         self.out = torch.empty((x.B, x.d), dtype=x.h.dtype, device=device)
         self.ws = torch.empty(int(gqa.lib.gqa_layer_decode_workspace_bytes(x.B, x.H, x.G, x.d_h,
                                                                              x.T_cap, gqa.GQA_BF16)),
@@ -437,8 +469,14 @@ class LayerDecode(QkvAppend):
                       + x.B * x.d * 2 + 2 * x.B * x.H * x.d_h + 2 * x.B * x.G * x.d_h) * e
         self.launches_per_step = 2 * ((x.B + 31) // 32) + 2
 
+    def _extra_weight_bytes(self):
+        x = self.x
+        return x.H * x.d_h * x.d * x.h.element_size()  # W_O
+
     def step(self, stream=None):
-        self.gqa.layer_decode_step(self.h, self.wq, self.wk, self.wv, self.wo, self.kc, self.vc,
+        k = self.i % self.n_sets
+        wq, wk, wv = self._next_set()
+        self.gqa.layer_decode_step(self.h, wq, wk, wv, self.wos[k], self.kc, self.vc,
                                    self.sl, out=self.out, seqlens_out=self.sl_out,
                                    workspace=self.ws, stream=stream)
 

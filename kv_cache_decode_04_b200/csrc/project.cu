@@ -13,8 +13,10 @@
 //
 // This is a skinny GEMM (B rows) bound by reading the weights once.  One CTA
 // owns 64 output columns of one of the three weights and streams them in
-// [128 rows x 64 columns] TMA tiles (128-byte swizzle) through a 6-stage
-// ring, together with the matching [32 sequences x 128] slice of h; four
+// [128 rows x 64 columns] TMA tiles (128-byte swizzle) through a 9-stage
+// ring (144 KB of weights in flight per SM: at this grid size the rate is
+// in-flight bytes over DRAM latency), with the matching [32 sequences x 128]
+// slice of h; four
 // warps split each tile's sixteen-row K-steps and run warp-level bf16 MMAs (B
 // padded to 16-row blocks), then the four partial sums are added in a fixed
 // order in shared memory, rounded once to bf16 and written.
@@ -28,7 +30,7 @@ namespace {
 
 constexpr int kNT = 64;                    // output columns per CTA
 constexpr int kKT = 128;                   // weight rows per stage
-constexpr int kStagesP = 6;
+constexpr int kStagesP = 9;
 constexpr int kCW = 4;                     // MMA warps
 constexpr int kThreadsP = (kCW + 1) * 32;  // + 1 TMA warp
 constexpr int kTileB = kKT * kNT * 2;      // 16 KB of weights per stage
@@ -64,8 +66,10 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-    float *red = reinterpret_cast<float *>(sm + kStagesP * kStageB);  // [kCW][RB*16][kNT]
-    uint64_t *full = reinterpret_cast<uint64_t *>(red + kCW * RB * 16 * kNT);
+    // After the main loop the ring is idle and holds the warps' partial sums,
+    // [kCW][RB*16][kNT] floats.
+    float *red = reinterpret_cast<float *>(sm);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + kStagesP * kStageB);
     uint64_t *empty = full + kStagesP;
     int *abort_flag = reinterpret_cast<int *>(empty + kStagesP);
     volatile int *vabort = abort_flag;
@@ -86,6 +90,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         fence_barrier_init();
     }
     __syncthreads();
+    pdl_wait_primary();  // h and seqlens written by the kernels before this one are visible
 
     if (warp == kCW) {  // ---------------- TMA producer
         if (lane == 0) {
@@ -93,6 +98,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             tma_prefetch_desc(&tmh);
             const uint64_t pol = l2_policy_evict_first();
             const uint64_t pol_h = l2_policy_evict_last();  // h is read by every CTA
+            int issued = 0;
             for (int kt = 0; kt < n_kt; ++kt) {
                 const int s = kt % kStagesP;
                 const uint32_t ph = (kt / kStagesP) & 1;
@@ -106,7 +112,11 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 tma_load_2d(st, tm, &full[s], col0, kt * kKT, pol);
                 tma_load_2d(st + kTileB, &tmh, &full[s], kt * kKT, p.b0, pol_h);
                 tma_load_2d(st + kTileB + kHHalf, &tmh, &full[s], kt * kKT + 64, p.b0, pol_h);
+                issued = kt + 1;
             }
+            if (*vabort)  // let copies still in flight land before the ring is reused or freed
+                for (int kt = max(0, issued - kStagesP); kt < issued; ++kt)
+                    mbar_wait(&full[kt % kStagesP], (kt / kStagesP) & 1, p.timeout_ns);
         }
         return;
     }
@@ -161,6 +171,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     }
 
     // ---------------- fixed-order sum of the four K-slices, one rounding, write
+    // (the ring is reused: wait until every MMA warp is done with its last tile)
+    asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
     float *my = red + warp * RB * 16 * kNT;
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb)
@@ -207,7 +219,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 template <int RB>
 cudaError_t run_proj(const ProjParams &p, const CUtensorMap *tq, const CUtensorMap *tk, const CUtensorMap *tv,
                      const CUtensorMap *th, cudaStream_t st) {
-    const size_t smem = 1024 + (size_t)kStagesP * kStageB + (size_t)kCW * RB * 16 * kNT * 4 + 2 * kStagesP * 8 + 16;
+    const size_t smem = 1024 + (size_t)kStagesP * kStageB + 2 * kStagesP * 8 + 16;
+    static_assert((size_t)kCW * 2 * 16 * kNT * 4 <= (size_t)kStagesP * kStageB, "partials fit in the ring");
     static int set_for[64];  // largest shared-memory size set, per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -217,8 +230,17 @@ cudaError_t run_proj(const ProjParams &p, const CUtensorMap *tq, const CUtensorM
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) set_for[dev] = (int)smem;
     }
-    qkv_append_kernel<RB><<<p.nq + 2 * p.nk, kThreadsP, smem, st>>>(*tq, *tk, *tv, *th, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.nq + 2 * p.nk));
+    cfg.blockDim = dim3(kThreadsP);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];  // programmatic dependent: the prologue may overlap the previous kernel
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, qkv_append_kernel<RB>, *tq, *tk, *tv, *th, p);
 }
 
 }  // namespace
