@@ -30,6 +30,8 @@
 // MMA tile.
 // fp32 path: CUDA-core fp32 arithmetic throughout (no TF32).
 #include <atomic>
+#include <chrono>
+#include <random>
 
 #include "common.cuh"
 #include "decode_common.cuh"
@@ -57,6 +59,9 @@ using dec::DecodeParams;
 using dec::kHalfBytes;
 using dec::kSplitPMaxLen;
 using dec::kTile;
+using dec::publish_flag;
+using dec::publish_prefix;
+using dec::wait_flag;
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -116,8 +121,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
     pdl_wait_primary();  // inputs written by the kernels before this one are visible
     const int W = build_tile_prefix<kTile>(p, cu, scratch, blockIdx.x == 0);
-    if (blockIdx.x == 0)
-        for (int i = tid; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
+    publish_prefix(p, cu);
     pdl_launch_dependents();
 
     const long long C = gridDim.x;
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         la += __shfl_xor_sync(0xffffffffu, la, 2);
         lb += __shfl_xor_sync(0xffffffffu, lb, 1);
         lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-        const long long rec = (long long)blockIdx.x + bg;  // rpp = 1
+        const long long rec = (long long)blockIdx.x + bg;
         if (NSL == 1) {
             const int hl_a = mt * 16 + g8, hl_b = hl_a + 8;
             if (!dead && hl_a < p.r) {
@@ -342,6 +346,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     *reinterpret_cast<float2 *>(dst + nn * 8 + 2 * q4) = make_float2(o[nn][2], o[nn][3]);
                 if (q4 == 0) p.ws_ml[rec * p.r + hl_b] = make_float2(m_b, lb);
             }
+            __threadfence();
+            named_bar_sync(1, kCWarps * 32);
+            if (tid == 0 && !dead) publish_flag(&p.ws_flag[1 + rec], p.gen);
         } else {
             // rows g8 and g8+8 of this warp's head tile; rows >= RR are past H/G
             float *ra = red + ((sl * NMT + mt) * RR + g8) * ROWF;
@@ -389,7 +396,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     if (col == 0) p.ws_ml[rec * p.r + hl] = make_float2(M, L);
                 }
             }
+            __threadfence();
             named_bar_sync(1, kCWarps * 32);
+            if (tid == 0 && !dead) publish_flag(&p.ws_flag[1 + rec], p.gen);
         }
     }
 }
@@ -414,8 +423,7 @@ __global__ void __launch_bounds__(kThreadsF32)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_wait_primary();  // inputs written by the kernels before this one are visible
     const int W = build_tile_prefix<kTileF32>(p, cu, scratch, blockIdx.x == 0);
-    if (blockIdx.x == 0)
-        for (int i = tid; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
+    publish_prefix(p, cu);
     pdl_launch_dependents();
     const long long C = gridDim.x;
     const int u_begin = (int)((long long)blockIdx.x * W / C);
@@ -486,33 +494,34 @@ __global__ void __launch_bounds__(kThreadsF32)
         cursor_next(cu, p.B, p.G, c);
         const bool piece_end = (u + 1 == u_end) || (c.b * p.G + c.g != bg);
         if (piece_end) {
-            const long long rec = (long long)blockIdx.x + bg;  // rpp = 1
+            const long long rec = (long long)blockIdx.x + bg;
             for (int i = tid; i < p.r * D; i += blockDim.x) p.ws_o[rec * p.r * D + i] = st_o[i];
             for (int i = tid; i < p.r; i += blockDim.x)
                 p.ws_ml[rec * p.r + i] = make_float2(st_m[i], st_l[i]);
+            __threadfence();
             __syncthreads();
+            if (tid == 0) publish_flag(&p.ws_flag[1 + rec], p.gen);
         }
     }
 }
 
 // ----------------------------------------------------------------- combine
 
-// One CTA of NW warps per output row (b, i).  Warp w merges records w,
-// w + NW, ... of the row's segment (record index i = piece * RPP + slice),
-// issuing the loads of up to kCombBatch records at once and keeping a running
-// (max, sum, o); the warps' results are then merged in a fixed order
-// (deterministic results).  A record with m = -inf (a slice that saw no
-// position) adds nothing.  NW is 16, 8 or 4 (see run_combine).
+// One CTA of NW warps per output row (b, i).  It runs alongside the split
+// kernel (a programmatic dependent launched early) and waits only for what it
+// reads: the tile prefix, then each record of its segment, through the
+// completion flags the split kernel publishes.  Warp w merges records w,
+// w + NW, ... of the row's segment, issuing the loads of up to kCombBatch
+// records at once and keeping a running (max, sum, o); the warps' results are
+// then merged in a fixed order (deterministic results).  NW is 16, 8 or 4
+// (see run_combine).
 constexpr int kCombBatch = 8;
 
-template <int D, bool BF16_OUT, int RPP, int NW>
+template <int D, bool BF16_OUT, int NW>
 __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, int C) {
-    constexpr int kCombWarps = NW;
-    pdl_wait_primary();  // the split kernel's records are complete and visible
-    pdl_launch_dependents();  // the next decode's split kernel may start its prologue
     constexpr int PER = D / 32;
-    __shared__ float red_m[kCombWarps], red_l[kCombWarps];
-    __shared__ __align__(16) float red_o[kCombWarps][D];
+    __shared__ float red_m[NW], red_l[NW];
+    __shared__ __align__(16) float red_o[NW][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row = blockIdx.x;  // b*H + h
     const int b = (int)(row / p.H), h = (int)(row % p.H);
@@ -522,28 +531,40 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
 #pragma unroll
     for (int k = 0; k < PER; ++k) acc[k] = 0.f;
     float M = -INFINITY, L = 0.f;
+    bool ok = __all_sync(0xffffffffu, wait_flag(&p.ws_flag[0], p.gen, p.timeout_ns));  // tile prefix
     const int *cu = p.ws_cu;
-    const int ntb = (cu[b + 1] - cu[b]) / p.G;
+    const int ntb = ok ? (cu[b + 1] - cu[b]) / p.G : 0;
     if (ntb > 0) {
         const long long W = cu[p.B];
         const long long s0 = cu[b] + (long long)g * ntb, s1 = s0 + ntb;
         const int c_lo = (int)(((s0 + 1) * C - 1) / W);
         const int c_hi = (int)((s1 * C - 1) / W);
-        const int n = (c_hi - c_lo + 1) * RPP;
+        const int n = c_hi - c_lo + 1;
         // With fewer tiles than CTAs some shares are empty; those CTAs wrote no record.
         const bool may_skip = W < C;
-        for (int i0 = warp; i0 < n; i0 += kCombWarps * kCombBatch) {
+        auto has_record = [&](int i) {
+            const int c = c_lo + i;
+            return i < n && !(may_skip && (long long)c * W / C == (long long)(c + 1) * W / C);
+        };
+        for (int i0 = warp; i0 < n && ok; i0 += NW * kCombBatch) {
+#pragma unroll 1
+            for (int j = 0; j < kCombBatch; ++j) {  // the batch's records are complete
+                const int i = i0 + j * NW;
+                if (has_record(i))
+                    ok &= __all_sync(0xffffffffu, wait_flag(&p.ws_flag[1 + (long long)c_lo + i + bg], p.gen,
+                                                            p.timeout_ns));
+            }
+            if (!ok) break;
             float2 ml[kCombBatch];
             float v[kCombBatch][PER];
 #pragma unroll
             for (int j = 0; j < kCombBatch; ++j) {
-                const int i = i0 + j * kCombWarps;
-                const int c = c_lo + i / RPP;
+                const int i = i0 + j * NW;
                 ml[j] = make_float2(-INFINITY, 0.f);
 #pragma unroll
                 for (int k = 0; k < PER; ++k) v[j][k] = 0.f;
-                if (i >= n || (may_skip && (long long)c * W / C == (long long)(c + 1) * W / C)) continue;
-                const long long rec = ((long long)c + bg) * RPP + i % RPP;
+                if (!has_record(i)) continue;
+                const long long rec = (long long)c_lo + i + bg;
                 ml[j] = p.ws_ml[rec * p.r + hl];
                 const float *src = p.ws_o + (rec * p.r + hl) * D + lane * PER;
                 if constexpr (PER == 4) {
@@ -570,6 +591,7 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
             }
         }
     }
+    if (!ok && lane == 0) set_status(p.status, STATUS_TIMEOUT);
 #pragma unroll
     for (int k = 0; k < PER; ++k) red_o[warp][lane * PER + k] = acc[k];
     if (lane == 0) {
@@ -577,16 +599,17 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
         red_l[warp] = L;
     }
     __syncthreads();
+    pdl_launch_dependents();  // the next decode's split kernel may start its prologue
     if (warp != 0) return;
     float Mt = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kCombWarps; ++w) Mt = fmaxf(Mt, red_m[w]);
+    for (int w = 0; w < NW; ++w) Mt = fmaxf(Mt, red_m[w]);
     float Lt = 0.f;
 #pragma unroll
     for (int k = 0; k < PER; ++k) acc[k] = 0.f;
     if (Mt != -INFINITY) {
 #pragma unroll
-        for (int w = 0; w < kCombWarps; ++w) {
+        for (int w = 0; w < NW; ++w) {
             const float f = fast_exp2(red_m[w] - Mt);  // 0 for a warp that merged nothing
             Lt = fmaf(f, red_l[w], Lt);
 #pragma unroll
@@ -686,12 +709,9 @@ cudaError_t run_combine_nw(const DecodeParams &p, int ctas, cudaStream_t st) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (carveout_dev != dev) {
-        const int pct = (int)cudaSharedmemCarveoutMaxShared;
-        for (auto kern : {decode_combine<D, BF16_OUT, 1, NW>, decode_combine<D, BF16_OUT, 2, NW>,
-                          decode_combine<D, BF16_OUT, 4, NW>}) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
-            if (e != cudaSuccess) return e;
-        }
+        e = cudaFuncSetAttribute(decode_combine<D, BF16_OUT, NW>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         carveout_dev = dev;
     }
     cudaLaunchConfig_t cfg = {};
@@ -704,24 +724,32 @@ cudaError_t run_combine_nw(const DecodeParams &p, int ctas, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    switch (p.rpp) {
-        case 1: return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT, 1, NW>, p, ctas);
-        case 2: return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT, 2, NW>, p, ctas);
-        case 4: return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT, 4, NW>, p, ctas);
-        default: return cudaErrorInvalidValue;
-    }
+    return cudaLaunchKernelEx(&cfg, decode_combine<D, BF16_OUT, NW>, p, ctas);
 }
 
 template <int D, bool BF16_OUT>
 cudaError_t run_combine(const DecodeParams &p, int ctas, cudaStream_t st) {
-    // Records of one row: about (CTAs per segment + 1) pieces of rpp records.
+    // Records of one row: about CTAs per segment + 1.
     // Wide CTAs (16 warps, one per SM by registers) only when the rows are few
     // enough to fit one wave and have records for the extra warps.
     const long long segs = (long long)p.B * p.G, rows = (long long)p.B * p.H;
-    const long long recs = (((long long)ctas + segs - 1) / segs + 1) * p.rpp;
+    const long long recs = ((long long)ctas + segs - 1) / segs + 1;
     if (rows <= 148 && recs > 16) return run_combine_nw<D, BF16_OUT, 16>(p, ctas, st);
     if (rows <= 3 * 148 && recs > 8) return run_combine_nw<D, BF16_OUT, 8>(p, ctas, st);
     return run_combine_nw<D, BF16_OUT, 4>(p, ctas, st);
+}
+
+// Call generations for the completion flags: unique per call in this process
+// and started from a random 64-bit base, so that flags left in reused memory
+// (by this or another process) do not match a new call's generation.
+unsigned long long next_generation() {
+    static std::atomic<unsigned long long> gen{[] {
+        std::random_device rd;
+        const unsigned long long t =
+            (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+        return ((unsigned long long)rd() << 32 ^ (unsigned long long)rd()) ^ (t * 0x9E3779B97F4A7C15ull);
+    }()};
+    return gen.fetch_add(1, std::memory_order_relaxed) + 1;
 }
 
 }  // namespace
@@ -738,12 +766,12 @@ DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, i
     if (ctas > max_tiles) ctas = max_tiles;
     if (ctas < 1) ctas = 1;
     L.ctas = (int)ctas;
-    L.rpp = tc ? dec::tc_records_per_piece(r) : 1;
-    L.n_rec = L.rpp * (ctas + (long long)B * G);
+    L.n_rec = ctas + (long long)B * G;
     L.off_cu = 0;
     L.off_ml = align256((size_t)(B + 1) * 4);
     L.off_o = L.off_ml + align256((size_t)L.n_rec * r * sizeof(float2));
-    L.total = L.off_o + align256((size_t)L.n_rec * r * d_h * sizeof(float));
+    L.off_flag = L.off_o + align256((size_t)L.n_rec * r * d_h * sizeof(float));
+    L.total = L.off_flag + align256((size_t)(1 + L.n_rec) * sizeof(unsigned long long));
     return L;
 }
 
@@ -776,7 +804,8 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUt
     p.T_cap = a.T_cap;
     p.timeout_ns = a.timeout_ns;
     p.window = a.window;
-    p.rpp = L.rpp;
+    p.ws_flag = reinterpret_cast<unsigned long long *>(ws + L.off_flag);
+    p.gen = next_generation();
     cudaError_t e;
     if (a.dtype == GQA_BF16) {
         const int nmt = bf16_nmt(p.r);

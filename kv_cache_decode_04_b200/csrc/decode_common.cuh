@@ -4,11 +4,12 @@
 // llm-arch-kb, section 1: G key/value heads per sequence) are laid end to end
 // and cut into gridDim.x equal shares.  CTA c takes share c; a share may cover
 // the tail of one segment and the head of the next.  For each piece (the part
-// of one segment inside one share) the CTA emits rpp partial records
-// (running max m in log2 units, sum l, unnormalised o[d_h]) per query head at
-// record indices rpp*(c + segment) + [0, rpp): distinct for all pieces, since
-// two pieces with equal c + segment would need an earlier CTA to hold a later
-// segment.  A record whose slice saw no position has m = -inf, l = 0, o = 0.
+// of one segment inside one share) the CTA emits one partial record (running
+// max m in log2 units, sum l, unnormalised o[d_h]) per query head at record
+// index c + segment: distinct for all pieces, since two pieces with equal
+// c + segment would need an earlier CTA to hold a later segment.  Each record
+// and the tile prefix carry a completion flag, so the combine can start on a
+// segment as soon as its records exist.
 #pragma once
 
 #include "common.cuh"
@@ -33,8 +34,48 @@ struct DecodeParams {
     int B, H, G, r, T_cap;
     unsigned long long timeout_ns;
     int window;  // > 0: attend over the last `window` cached positions only
-    int rpp;     // records per piece: piece (c, segment) owns records rpp*(c+segment) + [0, rpp)
+    // Completion flags, [1 + records]: flag 0 = the tile prefix ws_cu, flag 1 + i
+    // = record i.  A flag holds the generation of the call that completed it.
+    unsigned long long *ws_flag;
+    unsigned long long gen;  // this call's generation (unique per call and process)
 };
+
+// Publishes a completion flag with release semantics at GPU scope.  Every
+// thread that wrote part of the flagged data has executed __threadfence()
+// and a barrier shared with the publishing thread before this call.
+__device__ __forceinline__ void publish_flag(unsigned long long *flag, unsigned long long gen) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(flag), "l"(gen) : "memory");
+}
+
+// Waits, for at most limit_ns, until *flag == gen (acquire at GPU scope, so
+// this thread's later loads see the flagged data).  False on time-out.
+__device__ __forceinline__ bool wait_flag(const unsigned long long *flag, unsigned long long gen,
+                                          unsigned long long limit_ns) {
+    auto load = [&]() {
+        unsigned long long v;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flag) : "memory");
+        return v;
+    };
+    if (load() == gen) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        for (int i = 0; i < 32; ++i) {
+            __nanosleep(64);
+            if (load() == gen) return true;
+        }
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// CTA 0 of a split kernel: writes the tile prefix for the combine and
+// publishes it.  Every thread of the block calls it.
+__device__ __forceinline__ void publish_prefix(const DecodeParams &p, const int *cu) {
+    if (blockIdx.x != 0) return;
+    for (int i = threadIdx.x; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) publish_flag(&p.ws_flag[0], p.gen);
+}
 
 __device__ __forceinline__ int clamp_len(int T, int T_cap) {
     return T < 0 ? 0 : (T > T_cap ? T_cap : T);
@@ -151,8 +192,6 @@ constexpr int kTcMinHeads = 16;
 
 bool tc_eligible(int r, int d_h, int B);
 size_t tc_smem_bytes(int d_h, int B);
-// Records the tcgen05 kernel writes per piece (one per token slice).
-int tc_records_per_piece(int r);
 // Launches the tcgen05 split kernel on `ctas` CTAs (one per SM).
 cudaError_t run_split_tc(const DecodeParams &p, const CUtensorMap *tmk, const CUtensorMap *tmv, int d_h, int ctas,
                          cudaStream_t st);

@@ -198,8 +198,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     pdl_wait_primary();  // inputs written by the kernels before this one are visible
     const int W = build_tile_prefix<kTT>(p, cu, scratch, blockIdx.x == 0, tb);  // syncs the block
-    if (blockIdx.x == 0)
-        for (int i = tid; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
+    publish_prefix(p, cu);
     pdl_launch_dependents();
     tc::fence_after();
     const uint32_t tmem = *tmem_slot;
@@ -558,12 +557,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int kk = 0; kk < NREP; ++kk) acc += xp[((kk * NSW + hb) * 32 + i) * 33 + lane];
                         dst0[(size_t)i * D + c * 32 + lane] = acc;
                     }
+                    if (c == D / 32 - 1) {  // last chunk: the (M, L) pairs too, then make all visible
+                        if (k == 0 && valid) p.ws_ml[rec * p.r + head] = make_float2(M, L);
+                        __threadfence();
+                    }
                     if (!ep_sync()) {
                         ok = false;
                         return false;
                     }
                 }
-                if (k == 0 && valid) p.ws_ml[rec * p.r + head] = make_float2(M, L);
+                if (warp == 0 && lane == 0) publish_flag(&p.ws_flag[1 + rec], p.gen);
             }
             return true;
         });
@@ -603,11 +606,6 @@ bool tc_eligible(int r, int d_h, int B) {
 }
 
 size_t tc_smem_bytes(int d_h, int B) { return d_h == 128 ? smem_tc<128>(B) : smem_tc<64>(B); }
-
-int tc_records_per_piece(int r) {
-    (void)r;
-    return 1;  // the slices of a piece are merged in the split kernel
-}
 
 cudaError_t run_split_tc(const DecodeParams &p, const CUtensorMap *tmk, const CUtensorMap *tmv, int d_h, int ctas,
                          cudaStream_t st) {

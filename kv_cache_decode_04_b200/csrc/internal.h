@@ -32,9 +32,8 @@ struct DecodeArgs {
 // Workspace layout, all offsets 256-byte aligned.
 struct DecodeLayout {
     int ctas;          // split CTAs of the first kernel
-    int rpp;           // partial records per piece
-    long long n_rec;   // partial records: rpp * (ctas + B*G)
-    size_t off_cu, off_ml, off_o, total;
+    long long n_rec;   // partial records: ctas + B*G
+    size_t off_cu, off_ml, off_o, off_flag, total;
 };
 
 DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, int num_sms,

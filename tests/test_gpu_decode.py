@@ -146,3 +146,33 @@ def test_long_context_decode_full(gqa, G):
                                 rows=heads)
         assert_strict(out[b, heads], ref, torch.bfloat16)
         del kb, vb
+
+
+@pytest.mark.parametrize("H,G", [(32, 8), (32, 1)])
+def test_cuda_graph_replay_matches_eager(gqa, H, G):
+    """bench.py times decode steps replayed from a CUDA graph: the captured calls
+    (programmatic-dependent launches, completion flags from fresh call
+    generations at capture time) must give the eager calls' bits on every
+    replay, also with other work between replays."""
+    x = gi.decode_inputs(6, H, G, 128, 900, torch.bfloat16, seed=800 + G, ragged=(1, 900))
+    q, k, v = x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda()
+    sl = x.seqlens.to(torch.int32).cuda()
+    eager = gqa.decode(q, k, v, sl, x.scale).clone()
+    out = torch.empty_like(q)
+    ws = torch.empty(gqa.decode_workspace_bytes(6, H, G, 128, 900, q.dtype), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        gqa.decode(q, k, v, sl, x.scale, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    graph, s = torch.cuda.CUDAGraph(), torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=s):
+        for _ in range(3):
+            gqa.decode(q, k, v, sl, x.scale, out=out, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    for i in range(4):
+        out.zero_()
+        gqa.decode(q, k, v, sl, x.scale)  # another call (other workspace) between replays
+        graph.replay()
+        torch.cuda.synchronize()
+        gqa.get_status()
+        assert torch.equal(out, eager), "replay %d" % i
