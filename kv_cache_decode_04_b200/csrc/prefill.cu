@@ -210,8 +210,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t q_addr = smem_u32(sm + kOffQ), k_addr = smem_u32(sm + kOffK),
                            v_addr = smem_u32(sm + kOffV);
             bool issued = false, ok = true;
-            auto wait = [&](uint64_t *bar, uint32_t par) {
-                if (!ok || *vabort || !mbar_wait(bar, par, p.timeout_ns)) {
+            // The waits for P spin (test_wait) rather than suspend: a suspended thread
+            // resumed ~600 cycles after the softmax published P, and that delay sat on
+            // every tile's critical path.
+            auto wait = [&](uint64_t *bar, uint32_t par, bool spin = false) {
+                if (!ok || *vabort ||
+                    !(spin ? mbar_wait_spin(bar, par, p.timeout_ns) : mbar_wait(bar, par, p.timeout_ns))) {
                     if (ok) set_status(p.status, STATUS_TIMEOUT);
                     ok = false;
                     *vabort = 1;
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t ph = (j >> 1) & 1;
                     const int st2 = (j + 1) & 1;
                     const uint32_t ph2 = ((j + 1) >> 1) & 1;
-                    if (!wait(&v_full[st], ph) || !wait(&p_ready[0], j & 1)) break;
+                    if (!wait(&v_full[st], ph) || !wait(&p_ready[0], j & 1, true)) break;
                     tc::fence_after();
                     issue_pv(0, st, j > 0);
                     if (j + 1 < n_kv) {
@@ -265,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         issue_s(0, st2);
                         tc::commit(&s_full[0]);
                     }
-                    if (!wait(&p_ready[1], j & 1)) break;
+                    if (!wait(&p_ready[1], j & 1, true)) break;
                     tc::fence_after();
                     issue_pv(1, st, j > 0);
                     tc::commit(&v_empty[st]);
