@@ -103,3 +103,21 @@ def test_large_batches_near_the_shared_memory_bound(gqa, B):
     still fits the tensor-core kernel, B = 2400 takes the warp-MMA kernel."""
     x = gi.decode_inputs(B, 16, 1, 128, 40, torch.bfloat16, seed=770 + B, ragged=(0, 40))
     check(gqa, x)
+
+
+def test_one_workspace_alternating_shapes(gqa):
+    """Completion flags left in a workspace by one call never satisfy the next:
+    two shapes (the tensor-core and the warp-MMA split kernel) take turns on
+    one buffer, each call checked against the oracle."""
+    xa = gi.decode_inputs(3, 32, 1, 128, 700, torch.bfloat16, seed=780, seqlens=[700, 5, 333])
+    xb = gi.decode_inputs(4, 16, 4, 128, 500, torch.bfloat16, seed=781, seqlens=[1, 500, 64, 0])
+    refs = [oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale) for x in (xa, xb)]
+    dev = [(x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda(), x.seqlens.to(torch.int32).cuda(), x.scale)
+           for x in (xa, xb)]
+    need = max(gqa.decode_workspace_bytes(3, 32, 1, 128, 700), gqa.decode_workspace_bytes(4, 16, 4, 128, 500))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    for i in range(6):
+        q, k, v, sl, scale = dev[i % 2]
+        got = gqa.decode(q, k, v, sl, scale, workspace=ws)
+        gqa.get_status()
+        assert_close(got.cpu(), refs[i % 2], torch.bfloat16)
