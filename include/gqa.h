@@ -25,6 +25,10 @@
  *     a bounded wait that ran out) set bits of a device status word that
  *     gqa_get_status() reads and clears.  No kernel traps.
  *   - Results are deterministic: the same inputs and launch give the same bits.
+ *   - Kernels are launched as programmatic dependents: a call's set-up may
+ *     overlap the end of the work before it on `stream`, but no kernel reads
+ *     an input before that work has completed, so ordinary stream ordering
+ *     holds.  Calls can be captured in CUDA graphs.
  */
 #ifndef GQA_H
 #define GQA_H
@@ -96,13 +100,17 @@ GQA_API size_t gqa_decode_workspace_bytes(int B, int H, int G, int d_h, int T_ca
  *            T_b = 0 gives a zero output row.
  *   out      device, [B, H, d_h] dtype dt, 16-byte aligned
  *   workspace device, >= gqa_decode_workspace_bytes(...) bytes, 256-byte
- *            aligned; scratch for per-split partial results.
+ *            aligned; scratch for per-split partial results and their
+ *            completion flags.  Its contents need no initialisation.
  *   dt       GQA_BF16 (tensor-core scores and P.V, fp32 softmax/accumulate)
  *            or GQA_F32 (fp32 CUDA-core arithmetic throughout).
  *   Supported: d_h in {64, 128}; bf16 needs H/G <= 64.
  * Internally: a split-KV kernel over equal shares of the cache tiles (TMA
- * staged, fp32 online softmax per split) and a combine kernel that merges
- * the per-split (max, sum, partial output) triples exactly.
+ * staged, fp32 online softmax per split; warp-level MMAs for H/G <= 15,
+ * tcgen05 with S, P and O in tensor memory for 16 <= H/G <= 64) and a combine
+ * kernel that merges the per-split (max, sum, partial output) triples
+ * exactly, starting on a segment as soon as its splits have published their
+ * results.
  */
 GQA_API int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                const int32_t *seqlens, float scale, void *out, int B, int H,
