@@ -49,7 +49,6 @@
 // with the same stale maximum in numerator and denominator.
 #include "common.cuh"
 #include "decode_common.cuh"
-#include "exp2_fma.cuh"
 #include "internal.h"
 #include "tc.cuh"
 
@@ -456,8 +455,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
             // P = 2^(x - m) as bf16 pairs in this slice's columns of the S buffer,
-            // zeros in the other slices' columns; one exponential in four on the FMA
-            // pipe for full slices.  Short sequences also store P_lo = P - bf16(P).
+            // zeros in the other slices' columns (every exponential on the
+            // special-function unit).  Short sequences also store P_lo = P - bf16(P).
             const bool split = t.seq_len <= kSplitPMaxLen;
             const float mu = m == -INFINITY ? 0.f : m;  // no position seen yet: p = 0
             const uint64_t nm2 = f32x2_pack(-mu, -mu);
@@ -467,9 +466,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int e = 0; e < PCW; ++e) {
                 float x0, x1;
                 f32x2_unpack(f32x2_add(f32x2_pack(x[2 * e], x[2 * e + 1]), nm2), x0, x1);
-                const bool fma_pipe = !partial && !split && (e & 3) == 3;
-                const float p0 = fma_pipe ? exp2_fma(x0) : fast_exp2(x0);
-                const float p1 = fma_pipe ? exp2_fma(x1) : fast_exp2(x1);
+                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
                 rs2[e & 1] = f32x2_add(rs2[e & 1], f32x2_pack(p0, p1));
                 ph[e] = pack_bf16x2(p0, p1);
                 const float2 hv = unpack_bf16x2(ph[e]);

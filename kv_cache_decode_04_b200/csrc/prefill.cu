@@ -28,7 +28,6 @@
 #include <climits>
 
 #include "common.cuh"
-#include "exp2_fma.cuh"
 #include "gqa.h"
 #include "internal.h"
 #include "tc.cuh"
@@ -363,25 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2);
             const uint64_t nm2 = f32x2_pack(-mu, -mu);
             uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
-            if (!split_p && !diag && !lo_tile) {
-                // Off-diagonal tiles: one exponential in four on the FMA pipe
-                // (exp2_fma), the rest on the special-function unit.
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float x0, x1;
-                        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sr[c4][2 * e]),
-                                                          __uint_as_float(sr[c4][2 * e + 1])), sc2, nm2), x0, x1);
-                        const float p0 = (e & 3) == 3 ? exp2_fma(x0) : fast_exp2(x0);
-                        const float p1 = (e & 3) == 3 ? exp2_fma(x1) : fast_exp2(x1);
-                        rs2[e & 3] = f32x2_add(rs2[e & 3], f32x2_pack(p0, p1));
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tc::st16(tS + c4 * 16, pk);
-                }
-            } else if (!split_p) {
+            // Every exponential runs on the special-function unit: moving one in four to
+            // the FMA pipe (a Cody-Waite + polynomial exp2) was measured 6 % slower on
+            // this kernel, whose softmax is bound by instruction issue, not by that unit.
+            if (!split_p) {
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     uint32_t pk[16];
