@@ -8,7 +8,10 @@
 // in IEEE binary64 (ascending head order, correctly rounded division), then one
 // round-to-nearest-even to the storage type.  Every step is a correctly
 // rounded IEEE operation in a fixed order, so the result is bit-exact with
-// that definition.
+// that definition.  When r is a power of two the division is a multiplication
+// by 1/r: both are exact in binary64 here (the sums of bf16 or fp32 values are
+// far above the subnormal range), so the bits are the same and the FP64 pipe
+// is spared the division sequence.
 //
 // Streaming kernel: each thread produces 16 bytes of one output head from r
 // independent 16-byte loads (one per input head of its group); K and V are
@@ -68,7 +71,9 @@ __global__ void __launch_bounds__(256) meanpool_vec(const uint4 *__restrict__ wk
                                                     uint4 *ov, int r, long long n_vec,
                                                     long long out_vec, const float *wts, int sel) {
     const long long total = 2 * out_vec;
-    const double dr = (double)r;
+    const double dr = (double)r, inv_r = 1.0 / dr;
+    const bool pow2 = (r & (r - 1)) == 0;
+    auto mean = [&](double a) { return pow2 ? __dmul_rn(a, inv_r) : __ddiv_rn(a, dr); };
     const int H = (int)(r * (out_vec / n_vec));
     for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
@@ -87,8 +92,8 @@ __global__ void __launch_bounds__(256) meanpool_vec(const uint4 *__restrict__ wk
             uint32_t o[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const double a0 = MODE == MODE_MEAN ? __ddiv_rn(acc[2 * k], dr) : acc[2 * k];
-                const double a1 = MODE == MODE_MEAN ? __ddiv_rn(acc[2 * k + 1], dr) : acc[2 * k + 1];
+                const double a0 = MODE == MODE_MEAN ? mean(acc[2 * k]) : acc[2 * k];
+                const double a1 = MODE == MODE_MEAN ? mean(acc[2 * k + 1]) : acc[2 * k + 1];
                 o[k] = bf16_bits(a0) | (bf16_bits(a1) << 16);
             }
             st_stream((is_v ? ov : ok) + v, make_uint4(o[0], o[1], o[2], o[3]));
@@ -106,7 +111,7 @@ __global__ void __launch_bounds__(256) meanpool_vec(const uint4 *__restrict__ wk
             uint32_t *ow = &o.x;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                ow[k] = __float_as_uint(__double2float_rn(MODE == MODE_MEAN ? __ddiv_rn(acc[k], dr) : acc[k]));
+                ow[k] = __float_as_uint(__double2float_rn(MODE == MODE_MEAN ? mean(acc[k]) : acc[k]));
             st_stream((is_v ? ov : ok) + v, o);
         }
     }
@@ -118,7 +123,9 @@ __global__ void __launch_bounds__(256) meanpool_scalar(const void *wk, const voi
                                                        void *ov, int r, long long n,
                                                        long long out_n, const float *wts, int sel) {
     const long long total = 2 * out_n;
-    const double dr = (double)r;
+    const double dr = (double)r, inv_r = 1.0 / dr;
+    const bool pow2 = (r & (r - 1)) == 0;
+    auto mean = [&](double a) { return pow2 ? __dmul_rn(a, inv_r) : __ddiv_rn(a, dr); };
     const int H = (int)(r * (out_n / n));
     for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
@@ -137,7 +144,7 @@ __global__ void __launch_bounds__(256) meanpool_scalar(const void *wk, const voi
                     acc = __dadd_rn(acc, MODE == MODE_WEIGHTED ? __dmul_rn((double)wg[j], x) : x);
                 }
                 static_cast<__nv_bfloat16 *>(is_v ? ov : ok)[v] =
-                    __double2bfloat16(MODE == MODE_MEAN ? __ddiv_rn(acc, dr) : acc);
+                    __double2bfloat16(MODE == MODE_MEAN ? mean(acc) : acc);
             }
         } else {
             const float *src = static_cast<const float *>(is_v ? wv : wk) + g * r * n + e;
@@ -149,7 +156,7 @@ __global__ void __launch_bounds__(256) meanpool_scalar(const void *wk, const voi
                     acc = __dadd_rn(acc, MODE == MODE_WEIGHTED ? __dmul_rn((double)wg[j], x) : x);
                 }
                 static_cast<float *>(is_v ? ov : ok)[v] =
-                    __double2float_rn(MODE == MODE_MEAN ? __ddiv_rn(acc, dr) : acc);
+                    __double2float_rn(MODE == MODE_MEAN ? mean(acc) : acc);
             }
         }
     }
