@@ -48,9 +48,9 @@ ROW_WORKLOADS = ["tiny_decode_fp32", "llama2_70b_ragged_decode"] + \
 # no capture of its current kernel.
 NCU_TRAFFIC = {
     "llama2_7b_decode": 272122368,      # profiles/decode_split_llama2_7b.md (split kernel)
-    "long_ctx_decode_G1": 272365056,    # profiles/decode_split_tc_long_ctx_G1.md (tcgen05 split kernel)
-    "causal_prefill": 394518528,        # profiles/prefill_causal.md, half-length case x 4
-    "meanpool_init": 288346112,         # profiles/meanpool_init.md
+    "long_ctx_decode_G1": 273029376,    # profiles/decode_split_tc_long_ctx_G1.md (tcgen05 split kernel)
+    "causal_prefill": 397575168,        # profiles/prefill_causal.md, half-length case x 4
+    "meanpool_init": 289036800,         # profiles/meanpool_init.md
     "qkv_append_llama2_7b": 50488832,   # profiles/qkv_append_llama2_7b.md
 }
 
