@@ -47,7 +47,7 @@ ROW_WORKLOADS = ["tiny_decode_fp32", "llama2_70b_ragged_decode"] + \
 # captures of the current kernels (profiles/*.md); a workload missing here has
 # no capture of its current kernel.
 NCU_TRAFFIC = {
-    "llama2_7b_decode": 272122368,      # profiles/decode_split_llama2_7b.md (split kernel)
+    "llama2_7b_decode": 272493056,      # profiles/decode_split_llama2_7b.md (split kernel)
     "long_ctx_decode_G1": 273029376,    # profiles/decode_split_tc_long_ctx_G1.md (tcgen05 split kernel)
     "causal_prefill": 397575168,        # profiles/prefill_causal.md, half-length case x 4
     "meanpool_init": 289036800,         # profiles/meanpool_init.md
