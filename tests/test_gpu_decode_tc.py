@@ -121,3 +121,19 @@ def test_one_workspace_alternating_shapes(gqa):
         got = gqa.decode(q, k, v, sl, scale, workspace=ws)
         gqa.get_status()
         assert_close(got.cpu(), refs[i % 2], torch.bfloat16)
+
+
+def test_deterministic_across_streams(gqa):
+    """Every merge (slices of a piece, pieces of a segment) runs in a fixed
+    order, so repeated calls give the same bits, whatever the timing."""
+    x = gi.decode_inputs(5, 32, 1, 128, 3000, torch.bfloat16, seed=790, ragged=(1, 3000))
+    q, k, v = x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda()
+    sl = x.seqlens.to(torch.int32).cuda()
+    first = gqa.decode(q, k, v, sl, x.scale).clone()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        outs = [gqa.decode(q, k, v, sl, x.scale, stream=s) for _ in range(3)]
+    s.synchronize()
+    gqa.get_status()
+    for o in outs:
+        assert torch.equal(o, first)
