@@ -48,6 +48,51 @@ def test_meanpool_integer_coded(gqa):
         assert torch.equal(ok[g].double(), oracle.round_to(exp, torch.bfloat16).double())
 
 
+def _same_bits_or_both_nan(a, b):
+    nan = torch.isnan(a.float())
+    return torch.equal(nan, torch.isnan(b.float())) and torch.equal(bits(a)[~nan], bits(b)[~nan])
+
+
+def _bf16_mix(kind, H, n, seed):
+    """bf16 [H, n] inputs over the whole bf16 range, by kind."""
+    gen = torch.Generator().manual_seed(seed)
+    z = torch.randn(H, n, generator=gen, dtype=torch.float64)
+    if kind == "wide":  # exponents spread over 2^-40 .. 2^40 per element: the sums round
+        x = z * torch.exp2(torch.randint(-40, 40, (H, n), generator=gen).double())
+    elif kind == "edge":  # exponent spreads of 0..15 per group, full mantissas, a few negatives
+        base = torch.randint(20, 200, (1, n), generator=gen)
+        ex = base + torch.randint(0, 16, (H, n), generator=gen)
+        mant = torch.randint(0, 128, (H, n), generator=gen).double()
+        mant[:, ::2] = 127
+        sign = torch.where(torch.rand(H, n, generator=gen, dtype=torch.float64) < 0.1, -1.0, 1.0)
+        x = sign * (1 + mant / 128) * torch.exp2(ex.double() - 127)
+    else:  # "special": zeros, subnormals, +-inf, NaN, near-overflow values, cancelling pairs
+        x = z.clone()
+        u = torch.rand(H, n, generator=gen, dtype=torch.float64)
+        x[u < 0.01] = 0.0
+        x[(u >= 0.01) & (u < 0.02)] = float("inf")
+        x[(u >= 0.02) & (u < 0.025)] = float("-inf")
+        x[(u >= 0.025) & (u < 0.03)] = float("nan")
+        x[(u >= 0.03) & (u < 0.04)] = 1e-39
+        x[(u >= 0.04) & (u < 0.05)] = 3.3e38
+        x[1::2, ::3] = -x[0::2, ::3][: x[1::2, ::3].shape[0]]
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("H,G", [(64, 8), (48, 4), (8, 8), (64, 1), (12, 4)])
+@pytest.mark.parametrize("kind", ["wide", "edge", "special"])
+def test_meanpool_extreme_values_bit_exact(gqa, H, G, kind):
+    """Exponent spreads that make the binary64 sums round, full mantissas,
+    zeros, subnormals, +-inf, NaN, near-overflow values and cancelling pairs:
+    every output keeps the bits of the binary64 mean (NaN stays NaN)."""
+    d_h, d = 16, 64
+    wk = _bf16_mix(kind, H, d_h * d, seed=H * 7 + G).view(H, d_h, d)
+    wv = _bf16_mix(kind, H, d_h * d, seed=H * 7 + G + 1).view(H, d_h, d)
+    ok, ov = run(gqa, wk, wv, G)
+    assert _same_bits_or_both_nan(ok, oracle.meanpool(wk, G))
+    assert _same_bits_or_both_nan(ov, oracle.meanpool(wv, G))
+
+
 def test_meanpool_unaligned_views(gqa):
     """Element offsets that break 16-byte alignment take the element-wise kernel."""
     H, G, d_h, d = 8, 2, 5, 7
