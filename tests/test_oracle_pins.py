@@ -412,6 +412,25 @@ def test_qkv_append_grows_cache_by_2Gdh_scalars_per_token():
     assert torch.equal(kc[0, :, 0], k[0]) and torch.equal(vc[1, :, 4], v[1])
 
 
+def test_qkv_append_values_are_the_head_split_projections():
+    """KB s1: q = h W_Q split into H heads of d_h (head i = columns i*d_h ..),
+    k and v = h W_K, h W_V split into G heads, each written at position T_b of
+    its own sequence and KV head; checked against an fp64 torch matmul."""
+    B, d, H, G, d_h, T = 3, 48, 6, 3, 8, 7
+    x = gi.qkv_inputs(B, d, H, G, d_h, T, seed=31, seqlens=[0, 3, 6])
+    q, k, v, kc, vc, sl, app = oracle.qkv_append(x.h, x.W_Q, x.W_K, x.W_V, x.k_cache, x.v_cache,
+                                                 x.seqlens)
+    h = x.h.double()
+    tol = dict(rtol=1e-12, atol=1e-12)
+    torch.testing.assert_close(q, (h @ x.W_Q.double()).view(B, H, d_h), **tol)
+    torch.testing.assert_close(k, (h @ x.W_K.double()).view(B, G, d_h), **tol)
+    torch.testing.assert_close(v, (h @ x.W_V.double()).view(B, G, d_h), **tol)
+    for b, t in enumerate([0, 3, 6]):
+        for g in range(G):
+            assert torch.equal(kc[b, g, t], k[b, g]) and torch.equal(vc[b, g, t], v[b, g])
+    assert sl.tolist() == [1, 4, 7]
+
+
 # ----------------------------------------------------------------- sliding window
 
 def _band_sdpa_prefill(x, W):
