@@ -520,3 +520,23 @@ def test_layer_step_with_identity_output_projection_is_the_attention():
                              sl2, d_h ** -0.5)
     assert torch.equal(out, oracle.round_to(attn, st).double().reshape(2, d))
     assert sl.tolist() == [4, 9]
+
+
+def test_layer_step_output_is_concatenated_heads_times_W_O():
+    """KB s2 / s3: the layer output is the H heads' attention outputs laid side
+    by side ([B, H*d_h], head i at columns i*d_h ..) times W_O [H*d_h, d]; a
+    non-square W_O fixes the orientation.  Checked with an fp64 torch matmul."""
+    B, H, G, d_h, d = 2, 4, 2, 16, 40
+    x = gi.qkv_inputs(B, d, H, G, d_h, 9, seed=32, seqlens=[2, 7])
+    W_O = (torch.randn(H * d_h, d, generator=torch.Generator().manual_seed(33)) * 0.1).to(torch.bfloat16)
+    out, sl = oracle.layer_decode_step(x.h, x.W_Q, x.W_K, x.W_V, W_O, x.k_cache, x.v_cache,
+                                       x.seqlens, d_h ** -0.5)
+    q, k, v, kc, vc, sl2, _ = oracle.qkv_append(x.h, x.W_Q, x.W_K, x.W_V, x.k_cache, x.v_cache,
+                                                x.seqlens)
+    st = torch.bfloat16
+    attn = oracle.gqa_decode(oracle.round_to(q, st), oracle.round_to(kc, st), oracle.round_to(vc, st),
+                             sl2, d_h ** -0.5)
+    concat = torch.cat([oracle.round_to(attn, st)[:, i].double() for i in range(H)], dim=1)
+    assert out.shape == (B, d)
+    torch.testing.assert_close(out, concat @ W_O.double(), rtol=1e-12, atol=1e-12)
+    assert sl.tolist() == [3, 8]
