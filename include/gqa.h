@@ -101,7 +101,14 @@ GQA_API size_t gqa_decode_workspace_bytes(int B, int H, int G, int d_h, int T_ca
  *   out      device, [B, H, d_h] dtype dt, 16-byte aligned
  *   workspace device, >= gqa_decode_workspace_bytes(...) bytes, 256-byte
  *            aligned; scratch for per-split partial results and their
- *            completion flags.  Its contents need no initialisation.
+ *            completion flags.  Its contents need no initialisation.  Its
+ *            first 256 bytes carry, from one call to the next, the generation
+ *            number the completion flags are compared against; the device
+ *            advances it on every call, so a call captured in a CUDA graph
+ *            and replayed many times (with inputs changed in place between
+ *            replays) never accepts flags an earlier replay left behind.  Do
+ *            not write the workspace between calls that share it; after a
+ *            call on it reports GQA_ERR_TIMEOUT, re-capture graphs that use it.
  *   dt       GQA_BF16 (tensor-core scores and P.V, fp32 softmax/accumulate)
  *            or GQA_F32 (fp32 CUDA-core arithmetic throughout).
  *   Supported: d_h in {64, 128}; bf16 needs H/G <= 64.

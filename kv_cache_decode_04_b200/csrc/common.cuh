@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libgqa is built for sm_100a only"
 #endif
@@ -204,6 +206,24 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 
 __device__ __forceinline__ void pdl_wait_primary() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ------------------------------------------------------------ host
+
+// Runs `set` (a kernel-attribute call; the attribute persists per device)
+// once per device and kernel, one instance per kernel through the Tag type.
+// Thread-safe; a failed call is retried next time.
+template <typename Tag, typename Set>
+cudaError_t once_per_device(Set set) {
+    static std::atomic<bool> done[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = dev >= 0 && dev < 64;
+    if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = set();
+    if (e == cudaSuccess && cached) done[dev].store(true, std::memory_order_release);
+    return e;
 }
 
 }  // namespace gqa

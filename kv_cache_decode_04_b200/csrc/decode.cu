@@ -120,8 +120,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         tma_prefetch_desc(&tmv);
     }
     pdl_wait_primary();  // inputs written by the kernels before this one are visible
+    const unsigned long long gen = dec::call_generation(p);
     const int W = build_tile_prefix<kTile>(p, cu, scratch, blockIdx.x == 0);
-    publish_prefix(p, cu);
+    publish_prefix(p, cu, gen);
     pdl_launch_dependents();
 
     const long long C = gridDim.x;
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
             __threadfence();
             named_bar_sync(1, kCWarps * 32);
-            if (tid == 0 && !dead) publish_flag(&p.ws_flag[1 + rec], p.gen);
+            if (tid == 0 && !dead) publish_flag(&p.ws_flag[1 + rec], gen);
         } else {
             // rows g8 and g8+8 of this warp's head tile; rows >= RR are past H/G
             float *ra = red + ((sl * NMT + mt) * RR + g8) * ROWF;
@@ -398,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
             __threadfence();
             named_bar_sync(1, kCWarps * 32);
-            if (tid == 0 && !dead) publish_flag(&p.ws_flag[1 + rec], p.gen);
+            if (tid == 0 && !dead) publish_flag(&p.ws_flag[1 + rec], gen);
         }
     }
 }
@@ -422,8 +423,9 @@ __global__ void __launch_bounds__(kThreadsF32)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_wait_primary();  // inputs written by the kernels before this one are visible
+    const unsigned long long gen = dec::call_generation(p);
     const int W = build_tile_prefix<kTileF32>(p, cu, scratch, blockIdx.x == 0);
-    publish_prefix(p, cu);
+    publish_prefix(p, cu, gen);
     pdl_launch_dependents();
     const long long C = gridDim.x;
     const int u_begin = (int)((long long)blockIdx.x * W / C);
@@ -500,7 +502,7 @@ __global__ void __launch_bounds__(kThreadsF32)
                 p.ws_ml[rec * p.r + i] = make_float2(st_m[i], st_l[i]);
             __threadfence();
             __syncthreads();
-            if (tid == 0) publish_flag(&p.ws_flag[1 + rec], p.gen);
+            if (tid == 0) publish_flag(&p.ws_flag[1 + rec], gen);
         }
     }
 }
@@ -521,6 +523,7 @@ template <int D, bool BF16_OUT, int NW>
 __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, int C) {
     constexpr int PER = D / 32;
     __shared__ float red_m[NW], red_l[NW];
+    __shared__ int red_bad[NW];
     __shared__ __align__(16) float red_o[NW][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row = blockIdx.x;  // b*H + h
@@ -531,7 +534,9 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
 #pragma unroll
     for (int k = 0; k < PER; ++k) acc[k] = 0.f;
     float M = -INFINITY, L = 0.f;
-    bool ok = __all_sync(0xffffffffu, wait_flag(&p.ws_flag[0], p.gen, p.timeout_ns));  // tile prefix
+    const unsigned long long gen = dec::call_generation(p);
+    const bool pre_ok = __all_sync(0xffffffffu, wait_flag(&p.ws_flag[0], gen, p.timeout_ns));  // tile prefix
+    bool ok = pre_ok;
     const int *cu = p.ws_cu;
     const int ntb = ok ? (cu[b + 1] - cu[b]) / p.G : 0;
     if (ntb > 0) {
@@ -551,7 +556,7 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
             for (int j = 0; j < kCombBatch; ++j) {  // the batch's records are complete
                 const int i = i0 + j * NW;
                 if (has_record(i))
-                    ok &= __all_sync(0xffffffffu, wait_flag(&p.ws_flag[1 + (long long)c_lo + i + bg], p.gen,
+                    ok &= __all_sync(0xffffffffu, wait_flag(&p.ws_flag[1 + (long long)c_lo + i + bg], gen,
                                                             p.timeout_ns));
             }
             if (!ok) break;
@@ -592,6 +597,7 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
         }
     }
     if (!ok && lane == 0) set_status(p.status, STATUS_TIMEOUT);
+    if (lane == 0) red_bad[warp] = (pre_ok ? 0 : 2) | (ok ? 0 : 1);
 #pragma unroll
     for (int k = 0; k < PER; ++k) red_o[warp][lane * PER + k] = acc[k];
     if (lane == 0) {
@@ -601,6 +607,34 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
     __syncthreads();
     pdl_launch_dependents();  // the next decode's split kernel may start its prologue
     if (warp != 0) return;
+    if (lane == 0) {
+        // Count this CTA as finished (its read of the header is behind it).  The
+        // last CTA of the grid stores this call's generation for the next call,
+        // or, if a wait of any CTA ran out, a header that fails its check, so
+        // that the next call starts from a fresh random generation rather than
+        // one that flags left by this call could match.  The count was zeroed
+        // before the prefix flag; a CTA that never saw that flag does not count
+        // itself (the grid then never completes the count) and invalidates the
+        // header directly.
+        int bad = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) bad |= red_bad[w];
+        if (bad & 2) {
+            p.ws_hdr[dec::HDR_CHECK] = 0ull;
+        } else {
+            __threadfence();
+            const unsigned long long prev = atomicAdd(&p.ws_hdr[dec::HDR_DONE], 1ull + (bad ? (1ull << 32) : 0ull));
+            if ((prev & 0xffffffffull) == (unsigned long long)gridDim.x - 1) {
+                __threadfence();
+                if (bad || (prev >> 32)) {
+                    p.ws_hdr[dec::HDR_CHECK] = 0ull;
+                } else {
+                    p.ws_hdr[dec::HDR_EPOCH] = gen;
+                    p.ws_hdr[dec::HDR_CHECK] = gen ^ dec::kHdrMagic;
+                }
+            }
+        }
+    }
     float Mt = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) Mt = fmaxf(Mt, red_m[w]);
@@ -700,20 +734,18 @@ cudaError_t run_f32(const DecodeParams &p, int ctas, cudaStream_t st) {
 }
 
 template <int D, bool BF16_OUT, int NW>
+struct CombineTag {};
+
+template <int D, bool BF16_OUT, int NW>
 cudaError_t run_combine_nw(const DecodeParams &p, int ctas, cudaStream_t st) {
     // The split kernels before it run with (nearly) all of an SM's shared
     // memory; asking for the same carveout here spares every call an L1/shared
     // memory reconfiguration of the SMs between the two kernels.
-    static int carveout_dev = -1;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = once_per_device<CombineTag<D, BF16_OUT, NW>>([] {
+        return cudaFuncSetAttribute(decode_combine<D, BF16_OUT, NW>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    (int)cudaSharedmemCarveoutMaxShared);
+    });
     if (e != cudaSuccess) return e;
-    if (carveout_dev != dev) {
-        e = cudaFuncSetAttribute(decode_combine<D, BF16_OUT, NW>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        carveout_dev = dev;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((long long)p.B * p.H));
     cfg.blockDim = dim3(NW * 32);
@@ -739,10 +771,11 @@ cudaError_t run_combine(const DecodeParams &p, int ctas, cudaStream_t st) {
     return run_combine_nw<D, BF16_OUT, 4>(p, ctas, st);
 }
 
-// Call generations for the completion flags: unique per call in this process
-// and started from a random 64-bit base, so that flags left in reused memory
-// (by this or another process) do not match a new call's generation.
-unsigned long long next_generation() {
+// Seeds for the completion-flag generation (see dec::call_generation), used
+// when a workspace's header is not valid: unique per call in this process and
+// started from a random 64-bit base, so that flags left in reused memory (by
+// this or another process) do not match.
+unsigned long long next_seed() {
     static std::atomic<unsigned long long> gen{[] {
         std::random_device rd;
         const unsigned long long t =
@@ -767,8 +800,9 @@ DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, i
     if (ctas < 1) ctas = 1;
     L.ctas = (int)ctas;
     L.n_rec = ctas + (long long)B * G;
-    L.off_cu = 0;
-    L.off_ml = align256((size_t)(B + 1) * 4);
+    L.off_hdr = 0;
+    L.off_cu = 256;
+    L.off_ml = L.off_cu + align256((size_t)(B + 1) * 4);
     L.off_o = L.off_ml + align256((size_t)L.n_rec * r * sizeof(float2));
     L.off_flag = L.off_o + align256((size_t)L.n_rec * r * d_h * sizeof(float));
     L.total = L.off_flag + align256((size_t)(1 + L.n_rec) * sizeof(unsigned long long));
@@ -805,7 +839,8 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUt
     p.timeout_ns = a.timeout_ns;
     p.window = a.window;
     p.ws_flag = reinterpret_cast<unsigned long long *>(ws + L.off_flag);
-    p.gen = next_generation();
+    p.ws_hdr = reinterpret_cast<unsigned long long *>(ws + L.off_hdr);
+    p.seed = next_seed();
     cudaError_t e;
     if (a.dtype == GQA_BF16) {
         const int nmt = bf16_nmt(p.r);

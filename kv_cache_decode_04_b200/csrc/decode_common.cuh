@@ -37,8 +37,36 @@ struct DecodeParams {
     // Completion flags, [1 + records]: flag 0 = the tile prefix ws_cu, flag 1 + i
     // = record i.  A flag holds the generation of the call that completed it.
     unsigned long long *ws_flag;
-    unsigned long long gen;  // this call's generation (unique per call and process)
+    // Workspace header (first 256 bytes): the generation of the last call that
+    // completed on this workspace and a check word, and the combine's count of
+    // finished CTAs.  See call_generation().
+    unsigned long long *ws_hdr;
+    // Generation to start from when the header is not valid (fresh memory):
+    // random per host call.
+    unsigned long long seed;
 };
+
+// Header words.
+enum { HDR_EPOCH = 0, HDR_CHECK = 1, HDR_DONE = 2 };
+constexpr unsigned long long kHdrMagic = 0x6a09e667f3bcc909ull;
+
+// This call's generation, the value its completion flags carry.  Derived on
+// the device, so a call replayed from a CUDA graph (whose kernel arguments are
+// frozen) still gets a new one every time:
+//   - the combine's last CTA of every call stores that call's generation in
+//     the header with a check word; the next call on the workspace uses it + 1,
+//     so every flag an earlier call left behind holds a smaller value;
+//   - a header that fails the check (memory never used by a decode call, or
+//     invalidated after a timed-out wait) gives the host's random seed.
+// The split kernel reads the header after griddepcontrol.wait, when the last
+// call's combine has completed; the combine reads it before any of its CTAs
+// can advance it (the advance waits for all of them).  Every thread of a
+// kernel computes the same value.
+__device__ __forceinline__ unsigned long long call_generation(const DecodeParams &p) {
+    const volatile unsigned long long *h = p.ws_hdr;
+    const unsigned long long e = h[HDR_EPOCH], c = h[HDR_CHECK];
+    return c == (e ^ kHdrMagic) ? e + 1 : p.seed;
+}
 
 // Publishes a completion flag with release semantics at GPU scope.  Every
 // thread that wrote part of the flagged data has executed __threadfence()
@@ -67,14 +95,17 @@ __device__ __forceinline__ bool wait_flag(const unsigned long long *flag, unsign
     }
 }
 
-// CTA 0 of a split kernel: writes the tile prefix for the combine and
-// publishes it.  Every thread of the block calls it.
-__device__ __forceinline__ void publish_prefix(const DecodeParams &p, const int *cu) {
+// CTA 0 of a split kernel: writes the tile prefix for the combine, zeroes the
+// combine's finished-CTA count, and publishes both with the prefix flag (every
+// combine CTA waits for that flag before it counts itself).  Every thread of
+// the block calls it.
+__device__ __forceinline__ void publish_prefix(const DecodeParams &p, const int *cu, unsigned long long gen) {
     if (blockIdx.x != 0) return;
     for (int i = threadIdx.x; i <= p.B; i += blockDim.x) p.ws_cu[i] = cu[i];
+    if (threadIdx.x == 0) p.ws_hdr[HDR_DONE] = 0ull;
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) publish_flag(&p.ws_flag[0], p.gen);
+    if (threadIdx.x == 0) publish_flag(&p.ws_flag[0], gen);
 }
 
 __device__ __forceinline__ int clamp_len(int T, int T_cap) {

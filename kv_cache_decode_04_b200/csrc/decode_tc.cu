@@ -196,8 +196,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc::fence_before();
     }
     pdl_wait_primary();  // inputs written by the kernels before this one are visible
+    const unsigned long long gen = call_generation(p);
     const int W = build_tile_prefix<kTT>(p, cu, scratch, blockIdx.x == 0, tb);  // syncs the block
-    publish_prefix(p, cu);
+    publish_prefix(p, cu, gen);
     pdl_launch_dependents();
     tc::fence_after();
     const uint32_t tmem = *tmem_slot;
@@ -563,7 +564,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         return false;
                     }
                 }
-                if (warp == 0 && lane == 0) publish_flag(&p.ws_flag[1 + rec], p.gen);
+                if (warp == 0 && lane == 0) publish_flag(&p.ws_flag[1 + rec], gen);
             }
             return true;
         });
@@ -581,18 +582,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 template <int D, int NSW>
+struct TcTag {};
+
+template <int D, int NSW>
 cudaError_t run(const DecodeParams &p, const CUtensorMap *tmk, const CUtensorMap *tmv, int ctas, cudaStream_t st) {
     const size_t smem = smem_tc<D>(p.B);
     auto kern = decode_split_tc<D, NSW>;
-    static int set_dev = -1;  // the attribute persists per device; set it (to the maximum) on first use
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    // the attribute persists per device; set it (to the maximum) on first use
+    cudaError_t e = once_per_device<TcTag<D, NSW>>(
+        [&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024); });
     if (e != cudaSuccess) return e;
-    if (set_dev != dev) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        set_dev = dev;
-    }
     return launch_pdl(kern, dim3(ctas), dim3(kTcThreads), smem, st, *tmk, *tmv, p);
 }
 

@@ -29,11 +29,14 @@ struct DecodeArgs {
     int window;      // >0: sliding window of the last `window` cached positions
 };
 
-// Workspace layout, all offsets 256-byte aligned.
+// Workspace layout, all offsets 256-byte aligned.  The first 256 bytes are a
+// header that carries the completion-flag generation from one call to the
+// next; it sits at offset 0 for every shape, so calls of different shapes can
+// share a workspace.
 struct DecodeLayout {
     int ctas;          // split CTAs of the first kernel
     long long n_rec;   // partial records: ctas + B*G
-    size_t off_cu, off_ml, off_o, off_flag, total;
+    size_t off_hdr, off_cu, off_ml, off_o, off_flag, total;
 };
 
 DecodeLayout decode_layout(int B, int H, int G, int d_h, int T_cap, int dtype, int num_sms,

@@ -461,6 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+struct PrefillTag {};
+
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const CUtensorMap *tmk,
                            const CUtensorMap *tmv, cudaStream_t st) {
     PrefillParams p = {};
@@ -477,11 +479,14 @@ cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const C
     p.timeout_ns = a.timeout_ns;
     const long long grid = (long long)p.n_qt * a.B * a.G * (p.r / 2);
     if (grid <= 0 || grid >= (1ll << 31)) return cudaErrorInvalidConfiguration;
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_causal_kernel);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split would not hold
-    e = cudaFuncSetAttribute(prefill_causal_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaError_t e = once_per_device<PrefillTag>([] {
+        cudaFuncAttributes fa;
+        cudaError_t r = cudaFuncGetAttributes(&fa, prefill_causal_kernel);
+        if (r != cudaSuccess) return r;
+        if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split would not hold
+        return cudaFuncSetAttribute(prefill_causal_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes);
+    });
     if (e != cudaSuccess) return e;
     prefill_causal_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(*tmq, *tmk, *tmv, p);
     return cudaGetLastError();

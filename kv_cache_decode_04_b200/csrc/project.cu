@@ -217,19 +217,17 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 }
 
 template <int RB>
+struct ProjTag {};
+
+template <int RB>
 cudaError_t run_proj(const ProjParams &p, const CUtensorMap *tq, const CUtensorMap *tk, const CUtensorMap *tv,
                      const CUtensorMap *th, cudaStream_t st) {
     const size_t smem = 1024 + (size_t)kStagesP * kStageB + 2 * kStagesP * 8 + 16;
     static_assert((size_t)kCW * 2 * 16 * kNT * 4 <= (size_t)kStagesP * kStageB, "partials fit in the ring");
-    static int set_for[64];  // largest shared-memory size set, per device
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = once_per_device<ProjTag<RB>>([&] {
+        return cudaFuncSetAttribute(qkv_append_kernel<RB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || set_for[dev] < (int)smem) {
-        e = cudaFuncSetAttribute(qkv_append_kernel<RB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) set_for[dev] = (int)smem;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.nq + 2 * p.nk));
     cfg.blockDim = dim3(kThreadsP);

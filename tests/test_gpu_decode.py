@@ -176,3 +176,71 @@ def test_cuda_graph_replay_matches_eager(gqa, H, G):
         torch.cuda.synchronize()
         gqa.get_status()
         assert torch.equal(out, eager), "replay %d" % i
+
+
+@pytest.mark.parametrize("H,G,d_h,dtype", [
+    (32, 8, 128, torch.bfloat16),   # warp-MMA split kernel (4 heads per group)
+    (32, 1, 128, torch.bfloat16),   # tcgen05 split kernel (32 heads per group)
+    (8, 2, 64, torch.float32),      # fp32 split kernel
+])
+def test_single_call_graph_replay_with_changing_inputs(gqa, H, G, d_h, dtype):
+    """One decode call captured in a CUDA graph and replayed once per step, as a
+    serving loop does: q and seqlens change in place before every replay, and
+    eager calls on the same workspace run between replays.  Each replay must
+    give, bit for bit, what an eager call on the same inputs gives.  (Frozen
+    kernel arguments must not let a replay accept the partial results its
+    previous replay left in the workspace.)"""
+    B, T = 6, 900
+    x = gi.decode_inputs(B, H, G, d_h, T, dtype, seed=850 + G, nan_pad=False)
+    q, k, v = x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda()
+    sl = x.seqlens.to(torch.int32).cuda()
+    out = torch.empty_like(q)
+    ws = torch.empty(gqa.decode_workspace_bytes(B, H, G, d_h, T, dtype), dtype=torch.uint8,
+                     device="cuda")
+    gqa.decode(q, k, v, sl, x.scale, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    graph, s = torch.cuda.CUDAGraph(), torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=s):
+        gqa.decode(q, k, v, sl, x.scale, out=out, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    gen = torch.Generator().manual_seed(851)
+    for i in range(8):
+        q.copy_(torch.randn(q.shape, generator=gen).to(dtype))
+        lens = torch.randint(0, T + 1, (B,), generator=gen, dtype=torch.int32)
+        if i % 3 == 0:
+            lens[0] = 0
+        sl.copy_(lens)
+        graph.replay()
+        got = out.clone()
+        ref = gqa.decode(q, k, v, sl, x.scale)  # its own workspace
+        if i % 2:  # an eager call on the graph's workspace between replays
+            other = gqa.decode(q, k, v, sl, x.scale * 0.5, workspace=ws)
+            ref2 = gqa.decode(q, k, v, sl, x.scale * 0.5)
+            torch.cuda.synchronize()
+            assert torch.equal(other, ref2), "eager call on the shared workspace, step %d" % i
+        torch.cuda.synchronize()
+        gqa.get_status()
+        assert torch.equal(got, ref), "replay %d" % i
+
+
+@pytest.mark.parametrize("fill", ["zeros", "random", "ones"])
+def test_workspace_initial_contents_do_not_matter(gqa, fill):
+    """The workspace needs no initialisation: fresh zeros, random bytes, or a
+    fill whose header words look like flags all give the same bits."""
+    x = gi.decode_inputs(4, 32, 8, 128, 500, torch.bfloat16, seed=860, ragged=(1, 500))
+    q, k, v = x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda()
+    sl = x.seqlens.to(torch.int32).cuda()
+    ref = gqa.decode(q, k, v, sl, x.scale)
+    n = gqa.decode_workspace_bytes(4, 32, 8, 128, 500, torch.bfloat16)
+    if fill == "zeros":
+        ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    elif fill == "ones":
+        ws = torch.full((n,), 1, dtype=torch.uint8, device="cuda")
+    else:
+        g = torch.Generator(device="cuda").manual_seed(861)
+        ws = torch.randint(0, 256, (n,), generator=g, dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        out = gqa.decode(q, k, v, sl, x.scale, workspace=ws)
+        gqa.get_status()
+        assert torch.equal(out, ref)

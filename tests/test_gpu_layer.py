@@ -1,30 +1,26 @@
 """Output projection (gqa_out_project) and the whole-layer decode step
 (gqa_layer_decode_step: append, attend, project) vs the fp64 oracle.
 
-The layer stores q and the attention output in bf16 between its steps; the
-oracle rounds at the same points, but from fp64 instead of fp32 values, so an
-element close to a rounding boundary can end one bf16 step (2^-8 relative)
-apart on the two sides.  The layer test therefore allows, on top of the bf16
-tolerance, two such steps per attention element carried through W_O:
-2 * 2^-8 * (|attn| @ |W_O|).  The steps themselves are tested without it.
+The layer stores q and the attention output in bf16 between its steps, and
+the oracle rounds at the same two points (from fp64 values instead of fp32
+ones).  Where the two sides land one bf16 step apart on an intermediate, the
+step carries through W_O; such flips are rare (the fp32 and fp64 values differ
+by ~1e-7 relative against a 2^-8 step) and of random sign, so their carry is
+far below the tolerance and no allowance is added: the layer is held to the
+same bound as the kernels it is made of, the strict normwise form at the
+benchmark shape.  A negative control checks that this bound is tight enough
+to catch a wrong layer: against an oracle layer whose W_O has two heads'
+blocks of rows swapped (a head-order mistake, planted on the host side), the
+same GPU output must fail it.
 """
 import pytest
 import torch
 
 import gqa_inputs as gi
 import oracle
-from parity import assert_close, assert_close_plus
+from parity import assert_close, assert_strict, errors
 
 pytestmark = pytest.mark.gpu
-
-
-def _carry(x, W_O, scale, window):
-    """2 * 2^-8 * (|attn| @ |W_O|): two bf16 steps of every attention element carried by W_O."""
-    q, k, v, kc, vc, sl, _ = oracle.qkv_append(x.h, x.W_Q, x.W_K, x.W_V, x.k_cache, x.v_cache, x.seqlens)
-    st = torch.bfloat16
-    attn = oracle.gqa_decode(oracle.round_to(q, st), oracle.round_to(kc, st), oracle.round_to(vc, st),
-                             sl, scale, window=window)
-    return 2 * 2.0 ** -8 * (attn.abs().reshape(x.B, -1) @ W_O.double().abs())
 
 
 @pytest.mark.parametrize("B,K,N", [(1, 128, 64), (16, 4096, 4096), (33, 256, 192), (20, 512, 640)])
@@ -53,18 +49,36 @@ def test_layer_decode_step_small(gqa, B, d, H, G, d_h, T, seqlens, window):
     ref, rsl = oracle.layer_decode_step(x.h, x.W_Q, x.W_K, x.W_V, W_O, x.k_cache, x.v_cache,
                                         x.seqlens, d_h ** -0.5, window=window)
     assert torch.equal(sl.cpu(), rsl)
-    assert_close_plus(out.cpu(), ref, torch.bfloat16, _carry(x, W_O, d_h ** -0.5, window))
+    # short caches give O(1) outputs, where bf16 storage alone exceeds 2e-3:
+    # the per-element form |d| <= 2e-3 + 1e-2 |ref|
+    assert_close(out.cpu(), ref, torch.bfloat16)
+
+
+def _swap_head_blocks(W_O, d_h, a, b):
+    w = W_O.clone()
+    w[a * d_h:(a + 1) * d_h], w[b * d_h:(b + 1) * d_h] = W_O[b * d_h:(b + 1) * d_h], W_O[a * d_h:(a + 1) * d_h]
+    return w
 
 
 def test_layer_decode_step_llama2_7b(gqa):
-    """B=16, d=4096, H=32, G=8, d_h=128, T_cap=4096, one free slot per sequence."""
+    """B=16, d=4096, H=32, G=8, d_h=128, T_cap=4096, one free slot per sequence:
+    strict bound (max abs <= 2e-3 and max abs / max |ref| <= 1e-2) on every
+    output, and the negative control."""
     x = gi.workload_inputs("qkv_append_llama2_7b")
     gen = torch.Generator().manual_seed(8)
     W_O = (torch.randn(4096, 4096, generator=gen) * 4096 ** -0.5).to(torch.bfloat16)
     out, sl = gqa.layer_decode_step(x.h.cuda(), x.W_Q.cuda(), x.W_K.cuda(), x.W_V.cuda(), W_O.cuda(),
                                     x.k_cache.cuda(), x.v_cache.cuda(), x.seqlens.cuda())
     gqa.get_status()
+    out = out.cpu()
     ref, rsl = oracle.layer_decode_step(x.h, x.W_Q, x.W_K, x.W_V, W_O, x.k_cache, x.v_cache,
                                         x.seqlens, 128 ** -0.5)
     assert torch.equal(sl.cpu(), rsl)
-    assert_close_plus(out.cpu(), ref, torch.bfloat16, _carry(x, W_O, 128 ** -0.5, 0))
+    assert_strict(out, ref, torch.bfloat16)
+    # negative control: the oracle layer with heads 0 and 1 of W_O swapped
+    bad, _ = oracle.layer_decode_step(x.h, x.W_Q, x.W_K, x.W_V, _swap_head_blocks(W_O, 128, 0, 1),
+                                      x.k_cache, x.v_cache, x.seqlens, 128 ** -0.5)
+    with pytest.raises(AssertionError):
+        assert_strict(out, bad, torch.bfloat16)
+    maxabs, normrel = errors(out, bad)
+    assert normrel > 2e-2, (maxabs, normrel)  # fails by a wide margin, not at the edge

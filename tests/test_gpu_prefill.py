@@ -9,7 +9,7 @@ import torch
 
 import gqa_inputs as gi
 import oracle
-from parity import assert_close
+from parity import assert_close, assert_rows, full_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -57,15 +57,16 @@ def test_prefill_last_row_matches_decode(gqa):
 
 
 def test_causal_prefill_full_workload(gqa):
-    """B=2, S=8192, H=64, G=8, d_h=128: rows at tile edges and random rows."""
+    """B=2, S=8192, H=64, G=8, d_h=128: 1,154 sampled rows (every tile edge of one
+    (b, head) and 1,024 random rows), strict form on every row whose output stays
+    below 0.5 in magnitude."""
     x = gi.workload_inputs("causal_prefill")
     got = run(gqa, x)
     assert torch.isfinite(got.float()).all()
     S, H = 8192, 64
-    gen = torch.Generator().manual_seed(11)
-    picks = [(0, 0, 0), (1, 8191, 63), (0, 127, 5), (0, 128, 9), (1, 4095, 33), (1, 4096, 40)]
-    for s in torch.randint(0, S, (160,), generator=gen).tolist():
-        picks.append((s % 2, s, int(torch.randint(0, H, (1,), generator=gen))))
+    picks = full_rows(S, H, seed=11, n_random=1024)
+    assert len(picks) >= 1024 + 128
     rows = [(b * S + s) * H + i for b, s, i in picks]
     ref = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, rows=rows)
-    assert_close(got.reshape(-1, 128)[rows], ref, torch.bfloat16)
+    n_strict = assert_rows(got.reshape(-1, 128)[rows], ref, torch.bfloat16)
+    assert n_strict >= 0.95 * len(rows), n_strict  # all but the first few positions

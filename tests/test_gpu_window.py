@@ -5,7 +5,7 @@ import torch
 
 import gqa_inputs as gi
 import oracle
-from parity import assert_close, assert_strict
+from parity import assert_close, assert_rows, assert_strict, full_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -43,18 +43,17 @@ def test_prefill_window(gqa, S, W):
 
 
 def test_prefill_window_4096_full_workload(gqa):
-    """B=2, S=8192, H=64, G=8 with a 4096-key window: sampled rows."""
+    """B=2, S=8192, H=64, G=8 with a 4096-key window: every tile edge of one
+    (b, head) and 1,024 random rows; strict form on rows below 0.5."""
     x = gi.workload_inputs("causal_prefill")
     out = gqa.prefill_causal(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.scale, window=4096).cpu()
     gqa.get_status()
     S, H = 8192, 64
-    gen = torch.Generator().manual_seed(12)
-    picks = [(0, 0, 0), (1, 8191, 63), (0, 4095, 7), (0, 4096, 8), (1, 4097, 9), (1, 6000, 31)]
-    for s in torch.randint(0, S, (120,), generator=gen).tolist():
-        picks.append((s % 2, s, int(torch.randint(0, H, (1,), generator=gen))))
+    picks = full_rows(S, H, seed=12, n_random=1024, b_edge=0, head_edge=9)
     rows = [(b * S + s) * H + i for b, s, i in picks]
     ref = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, rows=rows, window=4096)
-    assert_close(out.reshape(-1, 128)[rows], ref, torch.bfloat16)
+    n_strict = assert_rows(out.reshape(-1, 128)[rows], ref, torch.bfloat16)
+    assert n_strict >= 0.95 * len(rows), n_strict
 
 
 def test_decode_window_4096_ragged_workload(gqa):
