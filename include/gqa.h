@@ -24,6 +24,11 @@
  *   - Conditions only the device can see (a seqlens entry outside [0, T_cap],
  *     a bounded wait that ran out) set bits of a device status word that
  *     gqa_get_status() reads and clears.  No kernel traps.
+ *   - libgqa_debug.so is the same library built with device-side index
+ *     checks: before a kernel uses an index it derived (a cache row, a
+ *     partial-record slot, a head, a weight row) it checks that the index
+ *     stays inside its buffer; a failed check skips the access and sets a
+ *     status bit (GQA_ERR_INDEX from gqa_get_status).  Same ABI and results.
  *   - Results are deterministic: the same inputs and launch give the same bits.
  *   - Kernels are launched as programmatic dependents: a call's set-up may
  *     overlap the end of the work before it on `stream`, but no kernel reads
@@ -58,7 +63,8 @@ enum {
     GQA_ERR_CUDA = -4,        /* a CUDA runtime or driver call failed         */
     GQA_ERR_WORKSPACE = -5,   /* workspace missing or too small               */
     GQA_ERR_TIMEOUT = -6,     /* device: a bounded wait ran out               */
-    GQA_ERR_SEQLEN = -7       /* device: a seqlens entry was outside [0,T_cap] */
+    GQA_ERR_SEQLEN = -7,      /* device: a seqlens entry was outside [0,T_cap] */
+    GQA_ERR_INDEX = -8        /* device, debug build only: an index check failed */
 };
 
 /*
@@ -178,9 +184,12 @@ GQA_API int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v
  *   q    device, [B, S, H, d_h] bf16, 16-byte aligned
  *   k, v device, [B, S, G, d_h] bf16, 16-byte aligned
  *   out  device, [B, S, H, d_h] bf16, 16-byte aligned
- *   Supported: dt = GQA_BF16, d_h = 128, H/G even, scale > 0; any S >= 1.
+ *   Supported: dt = GQA_BF16, d_h in {64, 128}, any G | H (G = H is MHA,
+ *   G = 1 is MQA), scale > 0, any S >= 1.
  * Internally: tcgen05 tensor-core MMAs with fp32 accumulators in tensor
- * memory, TMA-fed shared-memory tiles, fp32 online softmax, P in bf16.
+ * memory, TMA-fed shared-memory tiles, fp32 online softmax, P in bf16.  One
+ * CTA takes 128 positions of two heads of a group (both read the same K/V
+ * tiles); with an odd H/G the last head of each group runs alone.
  */
 GQA_API int gqa_prefill_causal(const void *q, const void *k, const void *v, void *out,
                        int B, int S, int H, int G, int d_h, float scale,
@@ -303,9 +312,10 @@ GQA_API int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_
 
 /*
  * gqa_get_status -- synchronises `stream`, then reads and clears the device
- * status word: GQA_OK, GQA_ERR_SEQLEN or GQA_ERR_TIMEOUT (device-side
- * conditions of earlier calls on this device), or GQA_ERR_CUDA if the
- * synchronisation itself failed.
+ * status word: GQA_OK, GQA_ERR_SEQLEN, GQA_ERR_TIMEOUT or (debug build)
+ * GQA_ERR_INDEX (device-side conditions of earlier calls on this device; the
+ * most severe is returned), or GQA_ERR_CUDA if the synchronisation itself
+ * failed.
  */
 GQA_API int gqa_get_status(gqa_stream_t stream);
 

@@ -26,11 +26,14 @@ __all__ = ["decode", "decode_noalloc", "decode_workspace_bytes", "prefill_causal
            "qkv_append", "init_kv_heads", "out_project", "layer_decode_step",
            "kv_cache_bytes", "get_status", "GQAError", "LIB_PATH", "lib"]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqa.so")
+# GQA_LIB=debug selects libgqa_debug.so: the same kernels with device-side
+# index checks compiled in (a failed check sets GQA_ERR_INDEX in the status word).
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libgqa_debug.so" if os.environ.get("GQA_LIB") == "debug" else "libgqa.so")
 
 GQA_F32, GQA_BF16 = 0, 1
 _ERRORS = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGN", -4: "CUDA", -5: "WORKSPACE",
-           -6: "TIMEOUT", -7: "SEQLEN"}
+           -6: "TIMEOUT", -7: "SEQLEN", -8: "INDEX"}
 
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_kv_cache_bytes", "gqa_decode_workspace_bytes", "gqa_decode",
@@ -48,8 +51,10 @@ class GQAError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libgqa.so is not built (expected at %s); run "
-                          "`python kv_cache_decode_04_b200/build.py`" % LIB_PATH)
+        raise ImportError("%s is not built (expected at %s); run "
+                          "`python kv_cache_decode_04_b200/build.py`%s"
+                          % (os.path.basename(LIB_PATH), LIB_PATH,
+                             " --debug" if "debug" in os.path.basename(LIB_PATH) else ""))
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.gqa_kv_cache_bytes.argtypes = [i32, i32, i32, i32]

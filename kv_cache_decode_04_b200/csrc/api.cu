@@ -247,8 +247,7 @@ static int prefill_impl(const void *q, const void *k, const void *v, void *out, 
     if (!std::isfinite(scale) || !(scale > 0.f))
         return fail(GQA_ERR_INVALID, "prefill scale must be finite and positive");
     if (dt != GQA_BF16) return fail(GQA_ERR_UNSUPPORTED, "prefill supports bf16 only");
-    if (d_h != 128) return fail(GQA_ERR_UNSUPPORTED, "prefill supports d_h=128 only (got %d)", d_h);
-    if ((H / G) % 2 != 0) return fail(GQA_ERR_UNSUPPORTED, "prefill needs an even H/G (got %d)", H / G);
+    if (d_h != 64 && d_h != 128) return fail(GQA_ERR_UNSUPPORTED, "prefill d_h=%d (built: 64, 128)", d_h);
     if ((long long)B * S * H >= (1ll << 31)) return fail(GQA_ERR_UNSUPPORTED, "B*S*H must be below 2^31");
     if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(out, 16))
         return fail(GQA_ERR_ALIGN, "q, k, v and out must be 16-byte aligned");
@@ -338,7 +337,7 @@ static int init_heads_impl(const void *WK, const void *WV, void *WK_out, void *W
     int rc = device_info(&d_);
     if (rc) return rc;
     cudaError_t e = gqa::launch_init_heads(WK, WV, WK_out, WV_out, H, G, n, dt, mode, weights, select,
-                                           d_->num_sms, reinterpret_cast<cudaStream_t>(stream));
+                                           d_->num_sms, d_->status, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "init-heads launch");
     return GQA_OK;
 }
@@ -520,6 +519,7 @@ int gqa_get_status(gqa_stream_t stream) {
         e = cudaMemcpy(d->status, &zero, sizeof zero, cudaMemcpyHostToDevice);
         if (e != cudaSuccess) return fail_cuda(e, "clearing the status word");
     }
+    if (word & 4u) return fail(GQA_ERR_INDEX, "an index check of the debug build failed (the access was skipped)");
     if (word & 2u) return fail(GQA_ERR_TIMEOUT, "a device-side wait ran out of time");
     if (word & 1u) return fail(GQA_ERR_SEQLEN, "a seqlens entry was outside [0, T_cap] (clamped)");
     return GQA_OK;

@@ -23,10 +23,27 @@ namespace gqa {
 enum : unsigned {
     STATUS_SEQLEN = 1u,   // a seqlens entry was outside [0, T_cap]
     STATUS_TIMEOUT = 2u,  // a bounded wait ran out
+    STATUS_INDEX = 4u,    // an index check of the debug build failed (the access was skipped)
 };
 
 __device__ __forceinline__ void set_status(unsigned *status, unsigned bit) {
     if (status) atomicOr(status, bit);
+}
+
+// Index checks of the debug build (compiled with -DGQA_DEBUG, libgqa_debug.so):
+// `ok` is the condition that an index about to be used stays inside its
+// buffer; when it fails the status word gets STATUS_INDEX and the caller
+// skips the access.  Nothing traps.  In the release build the check is the
+// constant true and costs nothing.
+__device__ __forceinline__ bool index_ok(bool ok, unsigned *status) {
+#ifdef GQA_DEBUG
+    if (!ok) set_status(status, STATUS_INDEX);
+    return ok;
+#else
+    (void)ok;
+    (void)status;
+    return true;
+#endif
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -30,6 +30,7 @@
 // MMA tile.
 // fp32 path: CUDA-core fp32 arithmetic throughout (no TF32).
 #include <atomic>
+#include <cstdlib>
 #include <chrono>
 #include <random>
 
@@ -150,8 +151,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const int Tb = clamp_len(p.seqlens[c.b], p.T_cap);
                 const int start = Tb - attended_len(Tb, p);
                 const int row = (c.b * p.G + c.g) * p.T_cap + start + c.j * kTile;
+                // the tile starts inside its (b, g) segment of the cache
+                const bool row_ok = index_ok(c.b < p.B && c.g < p.G && start + c.j * kTile < p.T_cap, p.status);
 #pragma unroll
                 for (int h = 0; h < HALVES; ++h) {
+                    // (a skipped tile leaves the barrier short of its bytes: the
+                    // consumers' bounded wait then ends the CTA)
+                    if (!row_ok) break;
                     tma_load_2d(kdst + h * kHalfBytes, &tmk, &full[s], h * 64, row, pol);
                     tma_load_2d(vdst + h * kHalfBytes, &tmv, &full[s], h * 64, row, pol);
                 }
@@ -331,6 +337,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         lb += __shfl_xor_sync(0xffffffffu, lb, 1);
         lb += __shfl_xor_sync(0xffffffffu, lb, 2);
         const long long rec = (long long)blockIdx.x + bg;
+        const bool rec_ok = index_ok(rec < p.n_rec, p.status);
+        if (!rec_ok) dead = true;
         if (NSL == 1) {
             const int hl_a = mt * 16 + g8, hl_b = hl_a + 8;
             if (!dead && hl_a < p.r) {
@@ -454,9 +462,10 @@ __global__ void __launch_bounds__(kThreadsF32)
             }
         }
         const size_t base = ((size_t)bg * p.T_cap + t0) * D;
+        const bool seg_ok = index_ok(b < p.B && t0 >= 0 && t0 + n_valid <= p.T_cap, p.status);
         for (int i = tid; i < kTileF32 * D; i += blockDim.x) {
             const int row = i / D, col = i - row * D;
-            const bool ok = row < n_valid;
+            const bool ok = row < n_valid && seg_ok;
             Ks[row * KS + col] = ok ? p.k32[base + i] : 0.f;
             Vs[row * KS + col] = ok ? p.v32[base + i] : 0.f;
         }
@@ -497,12 +506,14 @@ __global__ void __launch_bounds__(kThreadsF32)
         const bool piece_end = (u + 1 == u_end) || (c.b * p.G + c.g != bg);
         if (piece_end) {
             const long long rec = (long long)blockIdx.x + bg;
-            for (int i = tid; i < p.r * D; i += blockDim.x) p.ws_o[rec * p.r * D + i] = st_o[i];
-            for (int i = tid; i < p.r; i += blockDim.x)
-                p.ws_ml[rec * p.r + i] = make_float2(st_m[i], st_l[i]);
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) publish_flag(&p.ws_flag[1 + rec], gen);
+            if (index_ok(rec < p.n_rec, p.status)) {
+                for (int i = tid; i < p.r * D; i += blockDim.x) p.ws_o[rec * p.r * D + i] = st_o[i];
+                for (int i = tid; i < p.r; i += blockDim.x)
+                    p.ws_ml[rec * p.r + i] = make_float2(st_m[i], st_l[i]);
+                __threadfence();
+                __syncthreads();
+                if (tid == 0) publish_flag(&p.ws_flag[1 + rec], gen);
+            }
         }
     }
 }
@@ -549,7 +560,8 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
         const bool may_skip = W < C;
         auto has_record = [&](int i) {
             const int c = c_lo + i;
-            return i < n && !(may_skip && (long long)c * W / C == (long long)(c + 1) * W / C);
+            return i < n && !(may_skip && (long long)c * W / C == (long long)(c + 1) * W / C) &&
+                   index_ok(c_lo >= 0 && (long long)c + bg < p.n_rec, p.status);
         };
         for (int i0 = warp; i0 < n && ok; i0 += NW * kCombBatch) {
 #pragma unroll 1
@@ -840,6 +852,14 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUt
     p.window = a.window;
     p.ws_flag = reinterpret_cast<unsigned long long *>(ws + L.off_flag);
     p.ws_hdr = reinterpret_cast<unsigned long long *>(ws + L.off_hdr);
+    p.n_rec = L.n_rec;
+#ifdef GQA_DEBUG
+    // Test hook of the debug build only: declare one record fewer than a call
+    // over full-length sequences writes (its highest record index is
+    // n_rec - 2: the last CTA's last piece), so the index check on that record
+    // fires; the skipped record would still have been inside the workspace.
+    if (getenv("GQA_DEBUG_DECLARE_FEWER_RECORDS")) p.n_rec = L.n_rec - 2;
+#endif
     p.seed = next_seed();
     cudaError_t e;
     if (a.dtype == GQA_BF16) {

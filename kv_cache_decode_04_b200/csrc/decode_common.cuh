@@ -28,6 +28,7 @@ struct DecodeParams {
     int *ws_cu;     // [B+1] tile prefix, written by CTA 0 of the split kernel
     float2 *ws_ml;  // [n_rec * r]: (max in log2 units, sum)
     float *ws_o;    // [n_rec * r * d_h]: unnormalised outputs
+    long long n_rec;  // records the workspace holds (the debug build's index checks)
     const float *k32, *v32;  // fp32 path only
     unsigned *status;
     float scale_log2;

@@ -252,10 +252,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint8_t *kdst = sm + Lay::OFF_RING + s * Lay::STAGE_BYTES;
                 uint8_t *vdst = kdst + Lay::KV_BYTES;
                 mbar_arrive_expect_tx(&full[s], Lay::STAGE_BYTES);
+                // the tile starts inside its (b, g) segment of the cache (a skipped
+                // tile leaves the barrier short: the bounded waits then end the CTA)
+                const bool row_ok = index_ok(t.b < p.B && t.g < p.G && row - t.bg * p.T_cap >= 0 &&
+                                                 row - t.bg * p.T_cap < p.T_cap,
+                                             p.status);
 #pragma unroll
                 for (int h = 0; h < HALVES; ++h)
 #pragma unroll
                     for (int r2 = 0; r2 < kTT / 64; ++r2) {
+                        if (!row_ok) continue;
                         tma_load_2d(kdst + h * kBox + r2 * kHalfBytes, &tmk, &full[s], h * 64, row + r2 * 64, pol);
                         tma_load_2d(vdst + h * kBox + r2 * kHalfBytes, &tmv, &full[s], h * 64, row + r2 * 64, pol);
                     }
@@ -537,7 +543,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const float wgt = m == -INFINITY ? 0.f : fast_exp2(m - M);
                 const long long rec = (long long)blockIdx.x + t.bg;
                 float *dst0 = p.ws_o + (rec * p.r + hb * 32) * D;
-                const int nrows = min(32, p.r - hb * 32);
+                // the debug build's check: a record past the workspace is not written
+                const int nrows = index_ok(rec < p.n_rec, p.status) ? min(32, p.r - hb * 32) : 0;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t orow[32];
@@ -556,7 +563,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         dst0[(size_t)i * D + c * 32 + lane] = acc;
                     }
                     if (c == D / 32 - 1) {  // last chunk: the (M, L) pairs too, then make all visible
-                        if (k == 0 && valid) p.ws_ml[rec * p.r + head] = make_float2(M, L);
+                        if (k == 0 && valid && nrows > 0) p.ws_ml[rec * p.r + head] = make_float2(M, L);
                         __threadfence();
                     }
                     if (!ep_sync()) {
@@ -564,7 +571,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         return false;
                     }
                 }
-                if (warp == 0 && lane == 0) publish_flag(&p.ws_flag[1 + rec], gen);
+                if (warp == 0 && lane == 0 && rec < p.n_rec) publish_flag(&p.ws_flag[1 + rec], gen);
             }
             return true;
         });

@@ -88,9 +88,9 @@ int set_error(int code, const char *msg);
 // Mean-pool init, and its select-one-head / weighted-average alternatives
 // (mode 0, 1, 2; weights [2H] device floats for mode 2, K's then V's).
 cudaError_t launch_meanpool(const void *wk, const void *wv, void *ok, void *ov, int H, int G,
-                            long long n, int dtype, int num_sms, cudaStream_t stream);
+                            long long n, int dtype, int num_sms, unsigned *status, cudaStream_t stream);
 cudaError_t launch_init_heads(const void *wk, const void *wv, void *ok, void *ov, int H, int G,
                               long long n, int dtype, int mode, const float *weights, int select,
-                              int num_sms, cudaStream_t stream);
+                              int num_sms, unsigned *status, cudaStream_t stream);
 
 }  // namespace gqa

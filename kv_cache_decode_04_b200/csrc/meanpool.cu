@@ -69,7 +69,8 @@ template <bool BF16, int MODE>
 __global__ void __launch_bounds__(256) meanpool_vec(const uint4 *__restrict__ wk,
                                                     const uint4 *__restrict__ wv, uint4 *ok,
                                                     uint4 *ov, int r, long long n_vec,
-                                                    long long out_vec, const float *wts, int sel) {
+                                                    long long out_vec, const float *wts, int sel,
+                                                    unsigned *status) {
     const long long total = 2 * out_vec;
     const double dr = (double)r, inv_r = 1.0 / dr;
     const bool pow2 = (r & (r - 1)) == 0;
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(256) meanpool_vec(const uint4 *__restrict__ wk
         const bool is_v = idx >= out_vec;
         const long long v = is_v ? idx - out_vec : idx;
         const long long g = v / n_vec, e = v - g * n_vec;
+        if (!index_ok(g * r + r <= H && (MODE != MODE_SELECT || sel < r), status)) continue;
         const uint4 *src = (is_v ? wv : wk) + (g * r) * n_vec + e;
         const float *wg = MODE == MODE_WEIGHTED ? wts + (is_v ? H : 0) + g * r : nullptr;
         if constexpr (MODE == MODE_SELECT) {  // one head of the group, unchanged
@@ -121,7 +123,8 @@ __global__ void __launch_bounds__(256) meanpool_vec(const uint4 *__restrict__ wk
 template <bool BF16, int MODE>
 __global__ void __launch_bounds__(256) meanpool_scalar(const void *wk, const void *wv, void *ok,
                                                        void *ov, int r, long long n,
-                                                       long long out_n, const float *wts, int sel) {
+                                                       long long out_n, const float *wts, int sel,
+                                                       unsigned *status) {
     const long long total = 2 * out_n;
     const double dr = (double)r, inv_r = 1.0 / dr;
     const bool pow2 = (r & (r - 1)) == 0;
@@ -132,6 +135,7 @@ __global__ void __launch_bounds__(256) meanpool_scalar(const void *wk, const voi
         const bool is_v = idx >= out_n;
         const long long v = is_v ? idx - out_n : idx;
         const long long g = v / n, e = v - g * n;
+        if (!index_ok(g * r + r <= H && (MODE != MODE_SELECT || sel < r), status)) continue;
         const float *wg = MODE == MODE_WEIGHTED ? wts + (is_v ? H : 0) + g * r : nullptr;
         double acc = 0.0;
         if constexpr (BF16) {
@@ -164,7 +168,8 @@ __global__ void __launch_bounds__(256) meanpool_scalar(const void *wk, const voi
 
 template <int MODE>
 cudaError_t launch_mode(const void *wk, const void *wv, void *ok, void *ov, int H, int G, long long n, bool bf16,
-                        bool aligned, int num_sms, const float *wts, int sel, cudaStream_t st) {
+                        bool aligned, int num_sms, const float *wts, int sel, unsigned *status,
+                        cudaStream_t st) {
     const int r = H / G;
     const int per_vec = bf16 ? 8 : 4;
     const long long out_elems = (long long)G * n;
@@ -177,12 +182,12 @@ cudaError_t launch_mode(const void *wk, const void *wv, void *ok, void *ov, int 
         auto kern = bf16 ? meanpool_vec<true, MODE> : meanpool_vec<false, MODE>;
         kern<<<(unsigned)blocks, threads, 0, st>>>(static_cast<const uint4 *>(wk), static_cast<const uint4 *>(wv),
                                                    static_cast<uint4 *>(ok), static_cast<uint4 *>(ov), r, n_vec,
-                                                   out_vec, wts, sel);
+                                                   out_vec, wts, sel, status);
     } else {
         long long blocks = (2 * out_elems + threads - 1) / threads;
         if (blocks > cap) blocks = cap;
         auto kern = bf16 ? meanpool_scalar<true, MODE> : meanpool_scalar<false, MODE>;
-        kern<<<(unsigned)blocks, threads, 0, st>>>(wk, wv, ok, ov, r, n, out_elems, wts, sel);
+        kern<<<(unsigned)blocks, threads, 0, st>>>(wk, wv, ok, ov, r, n, out_elems, wts, sel, status);
     }
     return cudaGetLastError();
 }
@@ -190,13 +195,13 @@ cudaError_t launch_mode(const void *wk, const void *wv, void *ok, void *ov, int 
 }  // namespace
 
 cudaError_t launch_meanpool(const void *wk, const void *wv, void *ok, void *ov, int H, int G, long long n,
-                            int dtype, int num_sms, cudaStream_t st) {
-    return launch_init_heads(wk, wv, ok, ov, H, G, n, dtype, 0, nullptr, 0, num_sms, st);
+                            int dtype, int num_sms, unsigned *status, cudaStream_t st) {
+    return launch_init_heads(wk, wv, ok, ov, H, G, n, dtype, 0, nullptr, 0, num_sms, status, st);
 }
 
 cudaError_t launch_init_heads(const void *wk, const void *wv, void *ok, void *ov, int H, int G, long long n,
                               int dtype, int mode, const float *weights, int select, int num_sms,
-                              cudaStream_t st) {
+                              unsigned *status, cudaStream_t st) {
     const bool bf16 = dtype == GQA_BF16;
     const bool aligned = ((reinterpret_cast<uintptr_t>(wk) | reinterpret_cast<uintptr_t>(wv) |
                            reinterpret_cast<uintptr_t>(ok) | reinterpret_cast<uintptr_t>(ov)) &
@@ -204,11 +209,11 @@ cudaError_t launch_init_heads(const void *wk, const void *wv, void *ok, void *ov
     if ((long long)G * n == 0) return cudaSuccess;
     switch (mode) {
         case MODE_SELECT:
-            return launch_mode<MODE_SELECT>(wk, wv, ok, ov, H, G, n, bf16, aligned, num_sms, weights, select, st);
+            return launch_mode<MODE_SELECT>(wk, wv, ok, ov, H, G, n, bf16, aligned, num_sms, weights, select, status, st);
         case MODE_WEIGHTED:
-            return launch_mode<MODE_WEIGHTED>(wk, wv, ok, ov, H, G, n, bf16, aligned, num_sms, weights, select, st);
+            return launch_mode<MODE_WEIGHTED>(wk, wv, ok, ov, H, G, n, bf16, aligned, num_sms, weights, select, status, st);
         default:
-            return launch_mode<MODE_MEAN>(wk, wv, ok, ov, H, G, n, bf16, aligned, num_sms, weights, select, st);
+            return launch_mode<MODE_MEAN>(wk, wv, ok, ov, H, G, n, bf16, aligned, num_sms, weights, select, status, st);
     }
 }
 

@@ -8,8 +8,11 @@
 // every key), so QK^T and PV are dense tensor-core contractions here.
 //
 // One CTA = 128 query positions x 2 query heads of the same group: both heads
-// read the same K/V tiles, which each load therefore serves twice.
-//   warp 8      TMA producer: Q tiles once, then [128 x 128] K and V tiles of
+// read the same K/V tiles, which each load therefore serves twice.  When H/G
+// is odd, the last head of each group gets a CTA of its own (one head; the
+// second softmax warpgroup idles), so any group size works, H/G = 1 (MHA)
+// included.
+//   warp 8      TMA producer: Q tiles once, then [128 x d_h] K and V tiles of
 //               the group through 2-stage rings (128-byte swizzle).
 //   warp 9      allocates 512 tensor-memory columns; one lane issues every
 //               tcgen05.mma:  S_h = Q_h K_j^T  (fp32 in TMEM, 128 cols each)
@@ -18,7 +21,8 @@
 //   warps 4-7   one TMEM lane), head 1.  While one group runs its softmax the
 //               tensor core works on the other head's MMAs.
 //   warps 10-11 idle (they complete the third warpgroup for the register split).
-// TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,384) O0, [384,512) O1.
+// d_h is 64 or 128 (a template parameter).
+// TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,256+d_h) O0, [384,384+d_h) O1.
 // P (bf16) overwrites the first 64 columns of its S block after S is read.
 // Online softmax in the base-2 domain; the running max is only moved (and O
 // rescaled in TMEM) when it grows by more than 8, so p <= 2^8: the result is
@@ -39,7 +43,6 @@ namespace {
 constexpr int kBM = 128;                 // query rows per tile
 constexpr int kBN = 128;                 // keys per KV tile
 constexpr int kHalf = 128 * 64 * 2;      // one [128 rows x 64 bf16] swizzled box
-constexpr int kTile = 2 * kHalf;         // [128 x 128] bf16
 constexpr int kThreads = 384;           // 3 warpgroups
 // Register split (setmaxnreg): the launch gives every thread kLaunchRegs; the
 // TMA/MMA warpgroup then drops to kLowRegs and the two softmax warpgroups rise
@@ -51,11 +54,19 @@ constexpr int kLowRegs = 136;
 constexpr int kHighRegs = 184;
 static_assert(2 * 128 * kHighRegs + 128 * kLowRegs <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
-constexpr int kOffQ = 0;                 // Q0, Q1
-constexpr int kOffK = 2 * kTile;         // K stages 0, 1
-constexpr int kOffV = 4 * kTile;         // V stages 0, 1
-constexpr int kOffBar = 6 * kTile;
-constexpr size_t kSmemBytes = 1024 + kOffBar + 256;
+
+// Shared memory of the d_h = D kernel: Q0, Q1, K stages 0-1, V stages 0-1
+// ([128 x D] bf16 tiles of D/64 swizzled boxes each), then the barriers.
+template <int D>
+struct PLay {
+    static constexpr int HALVES = D / 64;
+    static constexpr int TILE = HALVES * kHalf;  // [128 x D] bf16
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = 2 * TILE;
+    static constexpr int OFF_V = 4 * TILE;
+    static constexpr int OFF_BAR = 6 * TILE;
+    static constexpr size_t SMEM = 1024 + OFF_BAR + 256;
+};
 
 struct PrefillParams {
     void *out;
@@ -96,19 +107,62 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
     return r;
 }
 
+// 2^x for a pair of fp32 values on the FMA and integer pipes instead of the
+// special-function unit, which the exponentials of a tile would otherwise keep
+// as busy as the tensor core.  x = j + f with j = round(x) (the 1.5 * 2^23
+// rounding trick) and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial whose
+// coefficients are a Remez (minimax) fit of the relative error over that
+// interval, max relative error 7.5e-5 (P is rounded to bf16, 2^-9, after
+// this); 2^j enters as j added to the exponent field.  x is clamped at -125
+// first, so the exponent cannot underflow: x = -inf (a masked key) gives
+// 2^-125 instead of 0, which no bf16 P or fp32 row sum can tell apart.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+    float x0, x1;
+    f32x2_unpack(x2, x0, x1);
+    const uint64_t x = f32x2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+    const uint64_t t = f32x2_add(x, f32x2_pack(kRound, kRound));
+    const uint64_t j = f32x2_add(t, f32x2_pack(-kRound, -kRound));
+    float j0, j1;
+    f32x2_unpack(j, j0, j1);
+    const uint64_t f = f32x2_add(x, f32x2_pack(-j0, -j1));
+    uint64_t q = f32x2_fma(f, f32x2_pack(0.05517167f, 0.05517167f), f32x2_pack(0.24261113f, 0.24261113f));
+    q = f32x2_fma(q, f, f32x2_pack(0.69326097f, 0.69326097f));
+    q = f32x2_fma(q, f, f32x2_pack(0.99992806f, 0.99992806f));
+    float q0, q1, t0, t1;
+    f32x2_unpack(q, q0, q1);
+    f32x2_unpack(t, t0, t1);
+    // the low bits of t hold j (t = 1.5 * 2^23 + j); shifting them into the
+    // exponent field drops the 1.5 * 2^23 part, whose low 9 bits are zero
+    const int r0 = (int)(__float_as_uint(t0) << 23) + (int)__float_as_uint(q0);
+    const int r1 = (int)(__float_as_uint(t1) << 23) + (int)__float_as_uint(q1);
+    return f32x2_pack(__int_as_float(r0), __int_as_float(r1));
+}
+
+// Pairs, out of every 8 of a row's 64 score pairs per tile, whose 2^x runs on
+// the FMA pipe (exp2_poly_x2) instead of the special-function unit.
+#ifndef GQA_PREFILL_EXP_POLY_OF_8
+#define GQA_PREFILL_EXP_POLY_OF_8 0
+#endif
+constexpr int kExpPolyOf8 = GQA_PREFILL_EXP_POLY_OF_8;
+
 // Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64_t limit) {
     const bool ok = mbar_wait(bar, parity, limit);
     return __all_sync(0xffffffffu, ok);
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_causal_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv, const PrefillParams p) {
+    using Lay = PLay<D>;
+    constexpr int HALVES = Lay::HALVES, kTile = Lay::TILE;
+    constexpr int kOffQ = Lay::OFF_Q, kOffK = Lay::OFF_K, kOffV = Lay::OFF_V;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::OFF_BAR);
     uint64_t *bar_q = bars + 0;
     uint64_t *k_full = bars + 1;   // [2]
     uint64_t *k_empty = bars + 3;  // [2]
@@ -124,14 +178,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // work unit: heaviest query tiles (most KV tiles) first
-    const int pairs = p.r >> 1;
+    // work unit: heaviest query tiles (most KV tiles) first; heads 2u, 2u+1 of the
+    // group, or head r-1 alone when r is odd
+    const int pairs = (p.r + 1) >> 1;
     const int per_qt = p.B * p.G * pairs;
     const int qt = p.n_qt - 1 - (int)(blockIdx.x / per_qt);
     const int rem = (int)(blockIdx.x % per_qt);
     const int b = rem / (p.G * pairs);
     const int g = (rem / pairs) % p.G;
-    const int h0 = g * p.r + 2 * (rem % pairs);
+    const int pr = rem % pairs;
+    const int h0 = g * p.r + 2 * pr;
+    const int nh = min(2, p.r - 2 * pr);  // heads of this CTA (1 or 2)
+    // the debug build's check of the unit's indices (uniform over the CTA: all
+    // threads leave before any barrier or tensor memory is set up)
+    if (!index_ok(qt >= 0 && b < p.B && g < p.G && nh >= 1 && h0 + nh <= p.H, p.status)) return;
     const int s0 = qt * kBM;
     // KV tiles j_lo..qt: with a sliding window of W keys the tiles wholly below the
     // first row's window (keys < s0 - W + 1) are skipped.
@@ -171,9 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmv);
             const uint64_t pol_q = l2_policy_evict_first();
             const uint64_t pol_kv = l2_policy_evict_last();
-            mbar_arrive_expect_tx(bar_q, 2 * kTile);
-            for (int hh = 0; hh < 2; ++hh)
-                for (int half = 0; half < 2; ++half)
+            mbar_arrive_expect_tx(bar_q, nh * kTile);
+            for (int hh = 0; hh < nh; ++hh)
+                for (int half = 0; half < HALVES; ++half)
                     tma_load_4d(sm + kOffQ + hh * kTile + half * kHalf, &tmq, bar_q, half * 64, h0 + hh, s0,
                                 b, pol_q);
             for (int jj = 0; jj < n_kv; ++jj) {
@@ -186,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 mbar_arrive_expect_tx(&k_full[st], kTile);
-                for (int half = 0; half < 2; ++half)
+                for (int half = 0; half < HALVES; ++half)
                     tma_load_4d(sm + kOffK + st * kTile + half * kHalf, &tmk, &k_full[st], half * 64, g, j * kBN,
                                 b, pol_kv);
                 if (*vabort || !mbar_wait(&v_empty[st], ph ^ 1, p.timeout_ns)) {
@@ -195,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 mbar_arrive_expect_tx(&v_full[st], kTile);
-                for (int half = 0; half < 2; ++half)
+                for (int half = 0; half < HALVES; ++half)
                     tma_load_4d(sm + kOffV + st * kTile + half * kHalf, &tmv, &v_full[st], half * 64, g, j * kBN,
                                 b, pol_kv);
             }
@@ -205,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = tc::idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idesc_o = tc::idesc_bf16(128, 128, false, true);
+            constexpr uint32_t idesc_o = tc::idesc_bf16(128, D, false, true);
             const uint32_t q_addr = smem_u32(sm + kOffQ), k_addr = smem_u32(sm + kOffK),
                            v_addr = smem_u32(sm + kOffV);
             bool issued = false, ok = true;
@@ -227,10 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dq = tc::sdesc_sw128(q_addr, 16, 1024);
             const uint64_t dk = tc::sdesc_sw128(k_addr, 16, 1024);
             const uint64_t dv = tc::sdesc_sw128(v_addr, kHalf, 1024);
-            // S_h = Q_h K^T: 8 K-steps of 16 over d_h = 128 (two 64-wide swizzled halves)
+            // S_h = Q_h K^T: D/16 K-steps of 16 over d_h (64-wide swizzled boxes)
             auto issue_s = [&](int hh, int ks) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
                     tc::mma_ss(tmem + hh * 128, dq + ((hh * kTile) >> 4) + off, dk + ((ks * kTile) >> 4) + off,
                                idesc_s, kk > 0 ? 1u : 0u);
@@ -248,11 +308,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    dv + ((vs * kTile + kk * 2048) >> 4), idesc_o,
                                    (acc || ps > 0 || kk > 0) ? 1u : 0u);
             };
+            const bool two = nh == 2;
             if (wait(bar_q, 0) && wait(&k_full[0], 0)) {
                 issue_s(0, 0);
                 tc::commit(&s_full[0]);
-                issue_s(1, 0);
-                tc::commit(&s_full[1]);
+                if (two) {
+                    issue_s(1, 0);
+                    tc::commit(&s_full[1]);
+                }
                 tc::commit(&k_empty[0]);
                 issued = true;
                 for (int j = 0; j < n_kv && ok; ++j) {  // j counts visited tiles
@@ -268,13 +331,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         issue_s(0, st2);
                         tc::commit(&s_full[0]);
                     }
-                    if (!wait(&p_ready[1], j & 1, true)) break;
-                    tc::fence_after();
-                    issue_pv(1, st, j > 0);
+                    if (two) {
+                        if (!wait(&p_ready[1], j & 1, true)) break;
+                        tc::fence_after();
+                        issue_pv(1, st, j > 0);
+                    }
                     tc::commit(&v_empty[st]);
                     if (j + 1 < n_kv) {
-                        issue_s(1, st2);
-                        tc::commit(&s_full[1]);
+                        if (two) {
+                            issue_s(1, st2);
+                            tc::commit(&s_full[1]);
+                        }
                         tc::commit(&k_empty[st2]);
                     }
                 }
@@ -300,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         // first key this row may see under a sliding window (none below it)
         const int key_lo = p.window > 0 ? s0 + t - p.window + 1 : INT_MIN;
-        for (int jj = 0; jj < n_kv; ++jj) {
+        const int my_kv = hh < nh ? n_kv : 0;  // a one-head CTA's second warpgroup has no work
+        for (int jj = 0; jj < my_kv; ++jj) {
             const int j = j_lo + jj;  // KV tile index
             const bool aborted = __any_sync(0xffffffffu, *vabort != 0);  // warp-uniform
             if (aborted || !warp_wait(&s_full[hh], jj & 1, p.timeout_ns)) {
@@ -371,10 +439,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        float x0, x1;
-                        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sr[c4][2 * e]),
-                                                          __uint_as_float(sr[c4][2 * e + 1])), sc2, nm2), x0, x1);
-                        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                        const uint64_t x2 = f32x2_fma(f32x2_pack(__uint_as_float(sr[c4][2 * e]),
+                                                                 __uint_as_float(sr[c4][2 * e + 1])), sc2, nm2);
+                        float p0, p1;
+                        if ((e & 7) < kExpPolyOf8) {
+                            f32x2_unpack(exp2_poly_x2(x2), p0, p1);
+                        } else {
+                            float x0, x1;
+                            f32x2_unpack(x2, x0, x1);
+                            p0 = fast_exp2(x0);
+                            p1 = fast_exp2(x1);
+                        }
                         rs2[e & 3] = f32x2_add(rs2[e & 3], f32x2_pack(p0, p1));
                         pk[e] = pack_bf16x2(p0, p1);
                     }
@@ -410,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (rescale) {  // O was last written by the P.V of tile j-1, complete by now
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < D / 16; ++c) {
                     uint32_t orow[16];
                     tc::ld16(tO + c * 16, orow);
                     tc::wait_ld();
@@ -426,14 +501,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // epilogue: O / l -> bf16 -> out[b, s0 + t, h0 + hh, :]
         const bool go = __all_sync(0xffffffffu, ok && *vabort == 0);
-        if (go && warp_wait(o_done, 0, p.timeout_ns)) {
+        if (hh >= nh) {
+            // no head: nothing to store
+        } else if (go && warp_wait(o_done, 0, p.timeout_ns)) {
             tc::fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const int s = s0 + t;
             __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) +
-                                 (((size_t)b * p.S + s) * p.H + h0 + hh) * 128;
+                                 (((size_t)b * p.S + s) * p.H + h0 + hh) * D;
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < D / 16; ++c) {
                 uint32_t orow[16];
                 tc::ld16(tO + c * 16, orow);
                 tc::wait_ld();
@@ -461,7 +538,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+template <int D>
 struct PrefillTag {};
+
+template <int D>
+cudaError_t run_prefill(const PrefillParams &p, long long grid, const CUtensorMap *tmq, const CUtensorMap *tmk,
+                        const CUtensorMap *tmv, cudaStream_t st) {
+    constexpr size_t smem = PLay<D>::SMEM;
+    cudaError_t e = once_per_device<PrefillTag<D>>([] {
+        cudaFuncAttributes fa;
+        cudaError_t r = cudaFuncGetAttributes(&fa, prefill_causal_kernel<D>);
+        if (r != cudaSuccess) return r;
+        if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split would not hold
+        return cudaFuncSetAttribute(prefill_causal_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem);
+    });
+    if (e != cudaSuccess) return e;
+    prefill_causal_kernel<D><<<(unsigned)grid, kThreads, smem, st>>>(*tmq, *tmk, *tmv, p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const CUtensorMap *tmk,
                            const CUtensorMap *tmv, cudaStream_t st) {
@@ -477,19 +572,11 @@ cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap *tmq, const C
     p.n_qt = (a.S + kBM - 1) / kBM;
     p.window = a.window;
     p.timeout_ns = a.timeout_ns;
-    const long long grid = (long long)p.n_qt * a.B * a.G * (p.r / 2);
+    const long long grid = (long long)p.n_qt * a.B * a.G * ((p.r + 1) / 2);
     if (grid <= 0 || grid >= (1ll << 31)) return cudaErrorInvalidConfiguration;
-    cudaError_t e = once_per_device<PrefillTag>([] {
-        cudaFuncAttributes fa;
-        cudaError_t r = cudaFuncGetAttributes(&fa, prefill_causal_kernel);
-        if (r != cudaSuccess) return r;
-        if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // register split would not hold
-        return cudaFuncSetAttribute(prefill_causal_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemBytes);
-    });
-    if (e != cudaSuccess) return e;
-    prefill_causal_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(*tmq, *tmk, *tmv, p);
-    return cudaGetLastError();
+    if (a.d_h == 64) return run_prefill<64>(p, grid, tmq, tmk, tmv, st);
+    if (a.d_h == 128) return run_prefill<128>(p, grid, tmq, tmk, tmv, st);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace gqa

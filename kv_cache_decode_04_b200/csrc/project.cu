@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         const __nv_bfloat16 o = __float2bfloat16_rn(v);
         const int n = col0 + c;
         if (region == 0) {
+            if (!index_ok(n < p.out_ld, p.status)) continue;
             p.q_out[(size_t)b * p.out_ld + n] = o;
         } else {
             const int T = p.seqlens[b];
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 continue;
             }
             const int g = n / p.d_h, dim = n - g * p.d_h;
+            if (!index_ok(g < p.G, p.status)) continue;
             __nv_bfloat16 *cache = region == 1 ? p.k_cache : p.v_cache;
             cache[(((size_t)b * p.G + g) * p.T_cap + T) * p.d_h + dim] = o;
         }

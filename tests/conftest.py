@@ -20,8 +20,9 @@ def _load_build_module():
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size workloads")
-    # libgqa.so is a build product (not committed); make sure it matches the sources
-    _load_build_module().build()
+    # libgqa.so and libgqa_debug.so are build products (not committed); make sure
+    # they match the sources
+    _load_build_module().build_all()
 
 
 def cuda_ok():

@@ -20,10 +20,12 @@ def test_header_declares_the_binding_exports():
 
 
 def test_library_exports_every_declared_symbol():
-    lib = ctypes.CDLL(gqa.LIB_PATH)
-    for name in declared_functions():
-        assert hasattr(lib, name), name
-    assert lib.gqa_version() == 100
+    pkg = os.path.dirname(gqa.LIB_PATH)
+    for so in ("libgqa.so", "libgqa_debug.so"):  # release and index-checked builds
+        lib = ctypes.CDLL(os.path.join(pkg, so))
+        for name in declared_functions():
+            assert hasattr(lib, name), (so, name)
+        assert lib.gqa_version() == 100
 
 
 def test_kv_cache_bytes_matches_oracle_and_pages():
@@ -60,7 +62,7 @@ def test_decode_rejects_bad_arguments_on_host():
 def test_prefill_and_meanpool_reject_bad_arguments_on_host():
     L = gqa.lib
     assert L.gqa_prefill_causal(16, 16, 16, 16, 1, 8, 8, 3, 128, 0.1, gqa.GQA_BF16, None) == -1
-    assert L.gqa_prefill_causal(16, 16, 16, 16, 1, 8, 8, 2, 64, 0.1, gqa.GQA_BF16, None) == -2
+    assert L.gqa_prefill_causal(16, 16, 16, 16, 1, 8, 8, 2, 96, 0.1, gqa.GQA_BF16, None) == -2  # d_h not built
     assert L.gqa_prefill_causal(16, 16, 16, 16, 1, 8, 8, 2, 128, 0.1, gqa.GQA_F32, None) == -2
     assert L.gqa_prefill_causal(16, 16, 16, 16, 1, 0, 8, 2, 128, 0.1, gqa.GQA_BF16, None) == -1
     assert L.gqa_prefill_causal(16, 16, 16, 8, 1, 8, 8, 2, 128, 0.1, gqa.GQA_BF16, None) == -3

@@ -38,6 +38,38 @@ def test_prefill_small(gqa, B, S, H, G):
     assert_close(got, ref, torch.bfloat16)
 
 
+@pytest.mark.parametrize("B,S,H,G,d_h", [
+    (1, 300, 4, 4, 128),     # G = H: MHA, every CTA holds one head
+    (2, 200, 6, 6, 64),      # MHA at d_h = 64, ragged S
+    (1, 384, 6, 2, 128),     # r = 3: one pair and one lone head per group
+    (2, 257, 10, 2, 128),    # r = 5, ragged S
+    (1, 640, 8, 1, 64),      # G = 1: MQA at d_h = 64
+    (1, 128, 2, 1, 64),      # one CTA at d_h = 64
+    (2, 777, 8, 2, 64),      # r = 4 at d_h = 64, ragged S
+    (1, 1, 3, 1, 64),        # a single position, r = 3
+])
+def test_prefill_group_sizes_and_head_dims(gqa, B, S, H, G, d_h):
+    x = gi.prefill_inputs(B, S, H, G, d_h, torch.bfloat16, seed=S + 13 * H + d_h)
+    got = run(gqa, x)
+    ref = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale)
+    assert_close(got, ref, torch.bfloat16)
+
+
+@pytest.mark.parametrize("H,G,d_h", [(8, 2, 128), (6, 2, 64), (4, 1, 128)])
+def test_prefill_gqa_equals_mha_on_repeated_kv(gqa, H, G, d_h):
+    """The page's broadcast identity on the GPU: GQA prefill equals MHA prefill
+    (G = H) on K/V repeat-interleaved H/G times along the head axis, bit for
+    bit, since each query head sees the same K/V values in the same order."""
+    x = gi.prefill_inputs(1, 300, H, G, d_h, torch.bfloat16, seed=40 + H + d_h)
+    gqa_out = run(gqa, x)
+    r = H // G
+    xr = gi.PrefillInputs(x.q, x.k.repeat_interleave(r, dim=2).contiguous(),
+                          x.v.repeat_interleave(r, dim=2).contiguous(), x.scale, 1, 300, H, H, d_h)
+    mha_out = run(gqa, xr)
+    assert torch.equal(gqa_out, mha_out)
+    assert_close(gqa_out, oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale), torch.bfloat16)
+
+
 def test_prefill_deterministic(gqa):
     x = gi.prefill_inputs(1, 512, 8, 2, 128, torch.bfloat16, seed=3)
     assert torch.equal(run(gqa, x), run(gqa, x))
