@@ -410,6 +410,9 @@ class QkvAppend:
         self.sl = x.seqlens.to(device)
         self.q = torch.empty((x.B, x.H, x.d_h), dtype=x.h.dtype, device=device)
         self.sl_out = torch.empty_like(self.sl)
+        # split-K over every SM (the workspace holds the partial sums of split blocks)
+        self.pws = torch.empty(gqa.project_workspace_bytes((x.H + 2 * x.G) * x.d_h, x.d), dtype=torch.uint8,
+                               device=device)
         e = x.h.element_size()
         # weights read once, h read, q written, one k and one v row per KV head written
         self.bytes = (x.d * (x.H + 2 * x.G) * x.d_h + x.B * x.d + x.B * x.H * x.d_h
@@ -428,7 +431,7 @@ class QkvAppend:
     def step(self, stream=None):
         wq, wk, wv = self._next_set()
         self.gqa.qkv_append(self.h, wq, wk, wv, self.kc, self.vc, self.sl,
-                            q_out=self.q, seqlens_out=self.sl_out, stream=stream)
+                            q_out=self.q, seqlens_out=self.sl_out, stream=stream, workspace=self.pws)
 
     def config(self):
         x = self.x
@@ -469,7 +472,7 @@ class LayerDecode(QkvAppend):
         self.wos = [wo.to(device) for _ in range(self.n_sets)]
         self.wo = self.wos[0]
         self.out = torch.empty((x.B, x.d), dtype=x.h.dtype, device=device)
-        self.ws = torch.empty(int(gqa.lib.gqa_layer_decode_workspace_bytes(x.B, x.H, x.G, x.d_h,
+        self.ws = torch.empty(int(gqa.lib.gqa_layer_decode_workspace_bytes(x.B, x.d, x.H, x.G, x.d_h,
                                                                              x.T_cap, gqa.GQA_BF16)),
                               dtype=torch.uint8, device=device)
         e = x.h.element_size()

@@ -245,12 +245,31 @@ GQA_API int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *
  *   k_cache, v_cache  device, [B, G, T_cap, d_h] bf16 (updated in place)
  *   seqlens           device, [B] int32 (read only)
  *   seqlens_out       device, [B] int32, or NULL; must not overlap seqlens
+ *   workspace         device, >= gqa_project_workspace_bytes((H + 2G) d_h, d)
+ *                     bytes, 256-byte aligned, or NULL (see below)
  *   Supported: dt = GQA_BF16, d a multiple of 128, d_h in {64, 128}.
+ * Internally: a skinny GEMM bound by reading the weights once.  Without a
+ * workspace, one CTA per 64 output columns; with one, the (column block,
+ * 128-row K tile) units are cut into equal shares, one CTA per SM, and the
+ * blocks split between CTAs are added up in a fixed order from fp32 partial
+ * sums in the workspace (same results on every call; they may differ from
+ * the workspace-free kernel's in the last bit, since the sums are grouped
+ * differently).  The workspace needs no initialisation; calls that run
+ * concurrently need separate workspaces.
  */
 GQA_API int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V,
                            void *q_out, void *k_cache, void *v_cache, const int32_t *seqlens,
                            int32_t *seqlens_out, int B, int d, int H, int G, int d_h, int T_cap,
-                           gqa_dtype dt, gqa_stream_t stream);
+                           gqa_dtype dt, void *workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/*
+ * gqa_project_workspace_bytes -- workspace the split-K projection kernel of
+ * gqa_qkv_append and gqa_out_project needs on the current device (it depends
+ * on the SM count) for ncols output columns (all three weights' for
+ * gqa_qkv_append, (H + 2G) d_h; N for gqa_out_project) and a reduction over d
+ * rows (K for gqa_out_project).  0 for a shape the kernels do not take.
+ */
+GQA_API size_t gqa_project_workspace_bytes(int ncols, int d);
 
 /*
  * gqa_init_kv_heads -- the mean-pool initialisation and the two alternatives
@@ -282,12 +301,14 @@ GQA_API int gqa_init_kv_heads(const void *WK, const void *WV, void *WK_out, void
  * section 2: the outputs concatenate across heads and are projected by W_O;
  * section 3: o.reshape(B, T, H*d_h) @ W_O), for one token per sequence:
  *     out[b, :] = x[b, :] W                 x [B, K], W [K, N], out [B, N]
- * bf16 in, fp32 accumulation, one rounding to bf16.  Same skinny-GEMM kernel
- * as gqa_qkv_append.  Supported: bf16, K a multiple of 128, N of 64; x and W
- * 16-byte aligned.
+ * bf16 in, fp32 accumulation, one rounding to bf16.  Same skinny-GEMM kernels
+ * as gqa_qkv_append, with the same optional workspace
+ * (>= gqa_project_workspace_bytes(N, K) bytes, or NULL).  Supported: bf16, K
+ * a multiple of 128, N of 64; x and W 16-byte aligned.
  */
 GQA_API int gqa_out_project(const void *x, const void *W, void *out, int B, int K, int N,
-                            gqa_dtype dt, gqa_stream_t stream);
+                            gqa_dtype dt, void *workspace, size_t workspace_bytes,
+                            gqa_stream_t stream);
 
 /*
  * gqa_layer_decode_step -- one decode step of a whole GQA attention layer
@@ -295,13 +316,14 @@ GQA_API int gqa_out_project(const void *x, const void *W, void *out, int B, int 
  * k/v appended at seqlens[b]), then gqa_decode_window over seqlens_out
  * (which includes the new token), then gqa_out_project of the attention
  * output with W_O into out [B, d].  q and the attention output are kept in
- * bf16 in the workspace between the steps.
+ * bf16 in the workspace between the steps; both projections use the split-K
+ * kernel, with their partial sums in the workspace too.
  *   W_O          device, [H*d_h, d] bf16
  *   seqlens_out  required: the lengths after the append
  *   workspace    >= gqa_layer_decode_workspace_bytes(...), 256-byte aligned
  * Other arguments as gqa_qkv_append and gqa_decode_window (window 0 = full).
  */
-GQA_API size_t gqa_layer_decode_workspace_bytes(int B, int H, int G, int d_h, int T_cap,
+GQA_API size_t gqa_layer_decode_workspace_bytes(int B, int d, int H, int G, int d_h, int T_cap,
                                                 gqa_dtype dt);
 GQA_API int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_K,
                                   const void *W_V, const void *W_O, void *k_cache,
@@ -334,7 +356,7 @@ GQA_API int gqa_selftest_wait_timeout(uint64_t limit_ns, int *waited, gqa_stream
 /* Reason for the last non-OK return on the calling thread ("" if none). */
 GQA_API const char *gqa_last_error_string(void);
 
-/* ABI version of this header: major * 100 + minor. */
+/* ABI version of this header: major * 100 + minor (1.01: optional projection workspaces). */
 GQA_API int gqa_version(void);
 
 #ifdef __cplusplus

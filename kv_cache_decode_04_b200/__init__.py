@@ -23,7 +23,7 @@ import os
 import torch
 
 __all__ = ["decode", "decode_noalloc", "decode_workspace_bytes", "prefill_causal", "meanpool_kv",
-           "qkv_append", "init_kv_heads", "out_project", "layer_decode_step",
+           "qkv_append", "init_kv_heads", "out_project", "project_workspace_bytes", "layer_decode_step",
            "kv_cache_bytes", "get_status", "GQAError", "LIB_PATH", "lib"]
 
 # GQA_LIB=debug selects libgqa_debug.so: the same kernels with device-side
@@ -39,7 +39,8 @@ _ERRORS = {-1: "INVALID", -2: "UNSUPPORTED", -3: "ALIGN", -4: "CUDA", -5: "WORKS
 EXPORTS = ("gqa_kv_cache_bytes", "gqa_decode_workspace_bytes", "gqa_decode",
            "gqa_decode_window", "gqa_decode_noalloc", "gqa_prefill_causal",
            "gqa_prefill_causal_window", "gqa_meanpool_kv", "gqa_init_kv_heads", "gqa_qkv_append",
-           "gqa_out_project", "gqa_layer_decode_workspace_bytes", "gqa_layer_decode_step",
+           "gqa_out_project", "gqa_project_workspace_bytes", "gqa_layer_decode_workspace_bytes",
+           "gqa_layer_decode_step",
            "gqa_selftest_wait_timeout", "gqa_get_status", "gqa_last_error_string", "gqa_version")
 
 
@@ -76,13 +77,15 @@ def _load():
     L.gqa_meanpool_kv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     L.gqa_meanpool_kv.restype = i32
     L.gqa_qkv_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
-                                 i32, vp]
+                                 i32, vp, sz, vp]
     L.gqa_qkv_append.restype = i32
     L.gqa_init_kv_heads.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, i32, i32, vp]
     L.gqa_init_kv_heads.restype = i32
-    L.gqa_out_project.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+    L.gqa_out_project.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, sz, vp]
     L.gqa_out_project.restype = i32
-    L.gqa_layer_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.gqa_project_workspace_bytes.argtypes = [i32, i32]
+    L.gqa_project_workspace_bytes.restype = sz
+    L.gqa_layer_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
     L.gqa_layer_decode_workspace_bytes.restype = sz
     L.gqa_layer_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, f32, i32, vp, i32, i32,
                                         i32, i32, i32, i32, i32, vp, sz, vp]
@@ -263,13 +266,29 @@ def init_kv_heads(wk, wv, G, mode="mean", head_weights=None, select=0, out_k=Non
     return out_k, out_v
 
 
+def project_workspace_bytes(ncols: int, d: int) -> int:
+    """Workspace of the split-K projection kernel: ncols output columns, d rows reduced."""
+    n = int(lib.gqa_project_workspace_bytes(int(ncols), int(d)))
+    if n == 0:
+        raise GQAError(-1, "unsupported projection shape: " + lib.gqa_last_error_string().decode())
+    return n
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+
+
 def qkv_append(h, W_Q, W_K, W_V, k_cache, v_cache, seqlens, q_out=None, seqlens_out=None,
-               stream=None):
+               stream=None, workspace=None):
     """One decode token: q = h W_Q, and h W_K, h W_V appended to the KV cache.
 
     h [B, d]; W_Q [d, H*d_h]; W_K, W_V [d, G*d_h]; k_cache, v_cache
     [B, G, T_cap, d_h] (written in place at position seqlens[b]); seqlens [B]
     int32.  Returns (q_out [B, H, d_h], seqlens_out [B] = seqlens + 1).
+    workspace (uint8, >= project_workspace_bytes((H + 2G) d_h, d)) selects the
+    split-K kernel that spreads the weights over every SM.
     """
     B, d = h.shape
     _, G, T_cap, d_h = k_cache.shape
@@ -285,13 +304,15 @@ def qkv_append(h, W_Q, W_K, W_V, k_cache, v_cache, seqlens, q_out=None, seqlens_
     rc = lib.gqa_qkv_append(_dev(h, "h"), _dev(W_Q, "W_Q"), _dev(W_K, "W_K"), _dev(W_V, "W_V"),
                             _dev(q_out, "q_out"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
                             _dev(seqlens, "seqlens"), _dev(seqlens_out, "seqlens_out"), B, d, H, G,
-                            d_h, T_cap, code, _stream(stream))
+                            d_h, T_cap, code, *_ws(workspace), _stream(stream))
     _check(rc)
     return q_out, seqlens_out
 
 
-def out_project(x, W, out=None, stream=None):
-    """out = x W for x [B, K] (e.g. the concatenated heads [B, H*d_h]) and W [K, N]."""
+def out_project(x, W, out=None, stream=None, workspace=None):
+    """out = x W for x [B, K] (e.g. the concatenated heads [B, H*d_h]) and W [K, N].
+
+    workspace (>= project_workspace_bytes(N, K)) selects the split-K kernel."""
     x2 = x.reshape(x.shape[0], -1)
     B, K = x2.shape
     if W.shape[0] != K:
@@ -300,7 +321,7 @@ def out_project(x, W, out=None, stream=None):
     if out is None:
         out = torch.empty((B, N), dtype=x.dtype, device=x.device)
     _check(lib.gqa_out_project(_dev(x2, "x"), _dev(W, "W"), _dev(out, "out"), B, K, N,
-                               _dtype_code(x), _stream(stream)))
+                               _dtype_code(x), *_ws(workspace), _stream(stream)))
     return out
 
 
@@ -320,7 +341,7 @@ def layer_decode_step(h, W_Q, W_K, W_V, W_O, k_cache, v_cache, seqlens, scale=No
         seqlens_out = torch.empty_like(seqlens)
     code = _dtype_code(h)
     if workspace is None:
-        n = int(lib.gqa_layer_decode_workspace_bytes(B, H, G, d_h, T_cap, code))
+        n = int(lib.gqa_layer_decode_workspace_bytes(B, d, H, G, d_h, T_cap, code))
         if n == 0:
             raise GQAError(-1, lib.gqa_last_error_string().decode())
         workspace = torch.empty(n, dtype=torch.uint8, device=h.device)

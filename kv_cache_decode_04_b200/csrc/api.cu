@@ -10,7 +10,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
+#include <random>
 
 #include "gqa.h"
 #include "internal.h"
@@ -83,6 +85,17 @@ uint64_t wait_timeout_ns() {
     return v;
 }
 
+// Tags for the split-K projections' block counters: nonzero, below 2^32, and
+// different from one call to the next.
+unsigned long long next_tag() {
+    static std::atomic<unsigned> t{(unsigned)std::random_device{}()};
+    unsigned v;
+    do {
+        v = t.fetch_add(1, std::memory_order_relaxed) + 1;
+    } while (v == 0);
+    return v;
+}
+
 int forced_splits() {
     const char *s = getenv("GQA_DECODE_CTAS");
     return s ? atoi(s) : 0;
@@ -137,7 +150,7 @@ int gqa::set_error(int code, const char *msg) { return fail(code, "%s", msg); }
 
 extern "C" {
 
-int gqa_version(void) { return 100; }
+int gqa_version(void) { return 101; }
 
 const char *gqa_last_error_string(void) { return t_err; }
 
@@ -353,9 +366,26 @@ int gqa_init_kv_heads(const void *WK, const void *WV, void *WK_out, void *WV_out
     return init_heads_impl(WK, WV, WK_out, WV_out, H, G, d_h, d, mode, head_weights, select, dt, stream);
 }
 
+size_t gqa_project_workspace_bytes(int ncols, int d) {
+    if (ncols <= 0 || d <= 0) return 0;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev)) return 0;
+    return gqa::proj_workspace_bytes(ncols, d, dev->num_sms);
+}
+
+static int check_proj_workspace(void *workspace, size_t bytes, int ncols, int d, int num_sms) {
+    if (!workspace) return GQA_OK;
+    const size_t need = gqa::proj_workspace_bytes(ncols, d, num_sms);
+    if (bytes < need)
+        return fail(GQA_ERR_WORKSPACE, "projection workspace of %zu bytes needed, %zu given", need, bytes);
+    if (misaligned(workspace, 256)) return fail(GQA_ERR_ALIGN, "workspace must be 256-byte aligned");
+    return GQA_OK;
+}
+
 int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V, void *q_out,
                    void *k_cache, void *v_cache, const int32_t *seqlens, int32_t *seqlens_out, int B, int d,
-                   int H, int G, int d_h, int T_cap, gqa_dtype dt, gqa_stream_t stream) {
+                   int H, int G, int d_h, int T_cap, gqa_dtype dt, void *workspace, size_t workspace_bytes,
+                   gqa_stream_t stream) {
     t_err[0] = 0;
     int rc = check_dims(B, H, G, d_h);
     if (rc) return rc;
@@ -374,6 +404,8 @@ int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *
         return fail(GQA_ERR_ALIGN, "weights and h must be 16-byte aligned");
     DeviceInfo *dev = nullptr;
     rc = device_info(&dev);
+    if (rc) return rc;
+    rc = check_proj_workspace(workspace, workspace_bytes, (H + 2 * G) * d_h, d, dev->num_sms);
     if (rc) return rc;
     CUtensorMap tq, tk, tv;
     {
@@ -415,13 +447,16 @@ int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *
     a.T_cap = T_cap;
     a.status = dev->status;
     a.timeout_ns = wait_timeout_ns();
+    a.workspace = workspace;
+    a.num_sms = dev->num_sms;
+    a.tag = next_tag();
     cudaError_t e = gqa::launch_qkv_append(a, &tq, &tk, &tv, &th, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "qkv_append launch");
     return GQA_OK;
 }
 
 int gqa_out_project(const void *x, const void *W, void *out, int B, int K, int N, gqa_dtype dt,
-                    gqa_stream_t stream) {
+                    void *workspace, size_t workspace_bytes, gqa_stream_t stream) {
     t_err[0] = 0;
     if (B <= 0 || K <= 0 || N <= 0) return fail(GQA_ERR_INVALID, "B, K and N must be positive");
     if (!x || !W || !out) return fail(GQA_ERR_INVALID, "null tensor pointer");
@@ -432,6 +467,8 @@ int gqa_out_project(const void *x, const void *W, void *out, int B, int K, int N
         return fail(GQA_ERR_ALIGN, "x and W must be 16-byte aligned");
     DeviceInfo *dev = nullptr;
     int rc = device_info(&dev);
+    if (rc) return rc;
+    rc = check_proj_workspace(workspace, workspace_bytes, N, K, dev->num_sms);
     if (rc) return rc;
     CUtensorMap tw, tx;
     {
@@ -448,7 +485,8 @@ int gqa_out_project(const void *x, const void *W, void *out, int B, int K, int N
         rc = make_tmap_bf16(&tx, x, 2, dims, strides, box);
         if (rc) return rc;
     }
-    cudaError_t e = gqa::launch_out_project(x, out, B, K, N, dev->status, wait_timeout_ns(), &tw, &tx,
+    cudaError_t e = gqa::launch_out_project(x, out, B, K, N, dev->status, wait_timeout_ns(), workspace,
+                                            dev->num_sms, next_tag(), &tw, &tx,
                                             reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "out_project launch");
     return GQA_OK;
@@ -456,10 +494,22 @@ int gqa_out_project(const void *x, const void *W, void *out, int B, int K, int N
 
 static size_t align256_host(size_t x) { return (x + 255) & ~size_t(255); }
 
-size_t gqa_layer_decode_workspace_bytes(int B, int H, int G, int d_h, int T_cap, gqa_dtype dt) {
+// The projections' split-K region of the layer workspace: the larger of the
+// Q/K/V projection's and W_O's (they run one after the other), or 0 when the
+// shape takes the column-block kernel.
+static size_t layer_proj_bytes(int d, int H, int G, int d_h) {
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev)) return 0;
+    const size_t a = gqa::proj_workspace_bytes((H + 2 * G) * d_h, d, dev->num_sms);
+    const size_t b = gqa::proj_workspace_bytes(d, H * d_h, dev->num_sms);
+    if (!a || !b) return 0;
+    return align256_host(a > b ? a : b);
+}
+
+size_t gqa_layer_decode_workspace_bytes(int B, int d, int H, int G, int d_h, int T_cap, gqa_dtype dt) {
     const size_t dec = gqa_decode_workspace_bytes(B, H, G, d_h, T_cap, dt);
-    if (!dec) return 0;
-    return 2 * align256_host((size_t)B * H * d_h * 2) + dec;
+    if (!dec || d <= 0) return 0;
+    return 2 * align256_host((size_t)B * H * d_h * 2) + layer_proj_bytes(d, H, G, d_h) + dec;
 }
 
 int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_K, const void *W_V, const void *W_O,
@@ -468,7 +518,7 @@ int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_K, const
                           gqa_dtype dt, void *workspace, size_t workspace_bytes, gqa_stream_t stream) {
     t_err[0] = 0;
     if (!seqlens_out) return fail(GQA_ERR_INVALID, "the layer step needs seqlens_out (lengths after the append)");
-    const size_t need = gqa_layer_decode_workspace_bytes(B, H, G, d_h, T_cap, dt);
+    const size_t need = gqa_layer_decode_workspace_bytes(B, d, H, G, d_h, T_cap, dt);
     if (!need) return decode_impl(nullptr, nullptr, nullptr, nullptr, scale, nullptr, B, H, G, d_h, T_cap, window, dt,
                                   nullptr, 0, stream);
     if (!workspace || workspace_bytes < need)
@@ -477,17 +527,20 @@ int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_K, const
     if (misaligned(workspace, 256)) return fail(GQA_ERR_ALIGN, "workspace must be 256-byte aligned");
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const size_t qbytes = align256_host((size_t)B * H * d_h * 2);
+    const size_t pbytes = layer_proj_bytes(d, H, G, d_h);
     void *q = ws, *attn = ws + qbytes;
+    void *pws = pbytes ? ws + 2 * qbytes : nullptr;  // split-K projections, when the shape allows them
+    uint8_t *dws = ws + 2 * qbytes + pbytes;
     // 1. q = h W_Q; k, v appended at seqlens[b]
     int rc = gqa_qkv_append(h, W_Q, W_K, W_V, q, k_cache, v_cache, seqlens, seqlens_out, B, d, H, G, d_h, T_cap,
-                            dt, stream);
+                            dt, pws, pbytes, stream);
     if (rc) return rc;
     // 2. attention over the cache including the new token
-    rc = decode_impl(q, k_cache, v_cache, seqlens_out, scale, attn, B, H, G, d_h, T_cap, window, dt,
-                     ws + 2 * qbytes, workspace_bytes - 2 * qbytes, stream);
+    rc = decode_impl(q, k_cache, v_cache, seqlens_out, scale, attn, B, H, G, d_h, T_cap, window, dt, dws,
+                     workspace_bytes - 2 * qbytes - pbytes, stream);
     if (rc) return rc;
     // 3. concatenated heads times W_O
-    return gqa_out_project(attn, W_O, out, B, H * d_h, d, dt, stream);
+    return gqa_out_project(attn, W_O, out, B, H * d_h, d, dt, pws, pbytes, stream);
 }
 
 int gqa_selftest_wait_timeout(uint64_t limit_ns, int *waited, gqa_stream_t stream) {

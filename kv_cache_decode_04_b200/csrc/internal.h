@@ -70,13 +70,20 @@ struct QkvArgs {
     int B, d, H, G, d_h, T_cap;
     unsigned *status;
     uint64_t timeout_ns;
+    void *workspace;         // null: one CTA per 64-column block; else the split-K kernel
+    int num_sms;
+    unsigned long long tag;  // nonzero, < 2^32: this call's tag for the split-K block counters
 };
 cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUtensorMap *tk,
                               const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t stream);
 
 cudaError_t launch_out_project(const void *x, void *out, int B, int K, int N, unsigned *status,
-                               uint64_t timeout_ns, const CUtensorMap *tw, const CUtensorMap *tx,
-                               cudaStream_t stream);
+                               uint64_t timeout_ns, void *workspace, int num_sms, unsigned long long tag,
+                               const CUtensorMap *tw, const CUtensorMap *tx, cudaStream_t stream);
+
+// Workspace of the split-K projection kernel for ncols output columns and a
+// reduction over d (0 when the shape is not supported).
+size_t proj_workspace_bytes(int ncols, int d, int num_sms);
 
 // One CTA waits on an mbarrier nothing arrives at, with the bounded wait.
 cudaError_t launch_wait_timeout_selftest(unsigned *status, uint64_t limit_ns, int *waited,

@@ -146,6 +146,13 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
 #endif
 constexpr int kExpPolyOf8 = GQA_PREFILL_EXP_POLY_OF_8;
 
+// 1: a tile's exponentials start from the running max before the tile's own
+// max is known (see the softmax); 0: max first, then the exponentials.
+#ifndef GQA_PREFILL_SPEC_MAX
+#define GQA_PREFILL_SPEC_MAX 0
+#endif
+constexpr bool kSpecMax = GQA_PREFILL_SPEC_MAX != 0;
+
 // Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64_t limit) {
     const bool ok = mbar_wait(bar, parity, limit);
@@ -405,83 +412,108 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[c][e]));
             const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
-            float alpha = 1.f;
-            bool rescale = false;
-            if (jj == 0) {
-                m = mx;  // -inf when a sliding window hides this tile from the row
-            } else {
-                const float mn = fmaxf(m, mx);
-                const bool need = mn > m + 8.f;
-                rescale = __any_sync(0xffffffffu, need);
-                if (need) {
-                    alpha = fast_exp2(m - mn);
-                    m = mn;
-                    l *= alpha;
-                }
-            }
             // P = 2^(s * scale_log2 - m) in bf16 pairs over the first 64 columns of
             // this S block; the exponent argument is formed two at a time (packed
             // fp32 FMA) and the row sum kept in four packed partial sums.
             // Rows of the first query tile see at most 128 keys, too few for the bf16
             // rounding of P to average out; there P is carried as P_hi + P_lo (two bf16
             // terms, about 16 significant bits), P_lo in columns 64..127.
-            // a row that has seen no key yet (m = -inf) has only -inf scores: p = 0
-            const float mu = m == -INFINITY ? 0.f : m;
+            // A row that has seen no key yet (m = -inf) has only -inf scores: p = 0.
+            // Returns the row sum of the unrounded p.
             const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2);
-            const uint64_t nm2 = f32x2_pack(-mu, -mu);
-            uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
-            // Every exponential runs on the special-function unit: moving one in four to
-            // the FMA pipe (a Cody-Waite + polynomial exp2) was measured 6 % slower on
-            // this kernel, whose softmax is bound by instruction issue, not by that unit.
-            if (!split_p) {
+            auto exp_pass = [&](float mrun) -> float {
+                const float mu = mrun == -INFINITY ? 0.f : mrun;
+                const uint64_t nm2 = f32x2_pack(-mu, -mu);
+                uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+                if (!split_p) {
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t pk[16];
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const uint64_t x2 = f32x2_fma(f32x2_pack(__uint_as_float(sr[c4][2 * e]),
-                                                                 __uint_as_float(sr[c4][2 * e + 1])), sc2, nm2);
-                        float p0, p1;
-                        if ((e & 7) < kExpPolyOf8) {
-                            f32x2_unpack(exp2_poly_x2(x2), p0, p1);
-                        } else {
-                            float x0, x1;
-                            f32x2_unpack(x2, x0, x1);
-                            p0 = fast_exp2(x0);
-                            p1 = fast_exp2(x1);
+                        for (int e = 0; e < 16; ++e) {
+                            const uint64_t x2 = f32x2_fma(f32x2_pack(__uint_as_float(sr[c4][2 * e]),
+                                                                     __uint_as_float(sr[c4][2 * e + 1])), sc2, nm2);
+                            float p0, p1;
+                            if ((e & 7) < kExpPolyOf8) {
+                                f32x2_unpack(exp2_poly_x2(x2), p0, p1);
+                            } else {
+                                float x0, x1;
+                                f32x2_unpack(x2, x0, x1);
+                                p0 = fast_exp2(x0);
+                                p1 = fast_exp2(x1);
+                            }
+                            rs2[e & 3] = f32x2_add(rs2[e & 3], f32x2_pack(p0, p1));
+                            pk[e] = pack_bf16x2(p0, p1);
                         }
-                        rs2[e & 3] = f32x2_add(rs2[e & 3], f32x2_pack(p0, p1));
-                        pk[e] = pack_bf16x2(p0, p1);
+                        tc::st16(tS + c4 * 16, pk);
                     }
-                    tc::st16(tS + c4 * 16, pk);
-                }
-            } else {  // first query tile: P_hi to columns 0..63, P_lo to 64..127
+                } else {  // first query tile: P_hi to columns 0..63, P_lo to 64..127
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
+                    for (int c4 = 0; c4 < 4; ++c4) {
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        uint32_t ph[4], pl[4];
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            uint32_t ph[4], pl[4];
 #pragma unroll
-                        for (int e1 = 0; e1 < 4; ++e1) {
-                            const int e = e4 * 4 + e1;
-                            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e]), p.scale_log2, -mu));
-                            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e + 1]), p.scale_log2, -mu));
-                            rs2[e1] = f32x2_add(rs2[e1], f32x2_pack(p0, p1));
-                            ph[e1] = pack_bf16x2(p0, p1);
-                            const float2 h = unpack_bf16x2(ph[e1]);
-                            pl[e1] = pack_bf16x2(p0 - h.x, p1 - h.y);
+                            for (int e1 = 0; e1 < 4; ++e1) {
+                                const int e = e4 * 4 + e1;
+                                const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e]), p.scale_log2, -mu));
+                                const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4][2 * e + 1]), p.scale_log2, -mu));
+                                rs2[e1] = f32x2_add(rs2[e1], f32x2_pack(p0, p1));
+                                ph[e1] = pack_bf16x2(p0, p1);
+                                const float2 h = unpack_bf16x2(ph[e1]);
+                                pl[e1] = pack_bf16x2(p0 - h.x, p1 - h.y);
+                            }
+                            tc::st4(tS + c4 * 16 + e4 * 4, ph);
+                            tc::st4(tS + 64 + c4 * 16 + e4 * 4, pl);
                         }
-                        tc::st4(tS + c4 * 16 + e4 * 4, ph);
-                        tc::st4(tS + 64 + c4 * 16 + e4 * 4, pl);
+                    }
+                }
+                float sum = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float a0, a1;
+                    f32x2_unpack(rs2[i], a0, a1);
+                    sum += a0 + a1;
+                }
+                return sum;
+            };
+            float alpha = 1.f;
+            bool rescale = false;
+            // With kSpecMax the running max m, which only moves when a tile's max
+            // exceeds it by more than 8, is used before this tile's max is known,
+            // so the exponentials need not wait for the max; a warp with a row
+            // whose max did move redoes the pass (its other rows recompute the same
+            // values).  Otherwise the max is settled first.
+            const bool spec = kSpecMax && jj > 0 && !split_p;
+            if (!spec) {
+                if (jj == 0) {
+                    m = mx;  // -inf when a sliding window hides this tile from the row
+                } else {
+                    const float mn = fmaxf(m, mx);
+                    const bool need = mn > m + 8.f;
+                    rescale = __any_sync(0xffffffffu, need);
+                    if (need) {
+                        alpha = fast_exp2(m - mn);
+                        m = mn;
+                        l *= alpha;
                     }
                 }
             }
-            float rs = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float a0, a1;
-                f32x2_unpack(rs2[i], a0, a1);
-                rs += a0 + a1;
+            float rs;
+#pragma unroll 1
+            for (int pass = 0;; ++pass) {
+                rs = exp_pass(m);
+                if (!spec || pass > 0) break;
+                const float mn = fmaxf(m, mx);
+                const bool need = mn > m + 8.f;  // also when m was -inf and mn is not
+                rescale = __any_sync(0xffffffffu, need);
+                if (!rescale) break;
+                if (need) {
+                    alpha = fast_exp2(m - mn);
+                    m = mn;
+                    l *= alpha;
+                }
+                tc::wait_st();
             }
             if (rescale) {  // O was last written by the P.V of tile j-1, complete by now
 #pragma unroll 1

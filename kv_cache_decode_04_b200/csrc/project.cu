@@ -218,6 +218,267 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         }
 }
 
+// ------------------------------------------------------------------------
+// Split-K variant for every SM.  The column-block kernel above gives each
+// 64-column block of the weights one CTA, which leaves SMs idle whenever
+// there are fewer blocks than SMs (96 for the Llama-2-7B Q/K/V projection, 64
+// for its W_O).  Here the units (column block cb, 128-row K tile kt), cb-major,
+// are laid end to end and cut into gridDim.x equal shares, one CTA per SM.  A
+// share's part of one block is a piece, with slot c + cb (distinct for all
+// pieces, as for the decode records).  A piece that covers its whole block is
+// rounded and stored directly; any other writes its fp32 partial sums to its
+// slot in the workspace and counts itself on the block's counter, and the
+// piece that completes the count adds the block's partials up in slot order
+// (the same order whichever piece finishes last: deterministic), rounds once
+// and stores.  Each MMA warp owns 16 of the block's 64 columns over all K
+// steps, so a warp's partial needs no reduction across warps.
+//
+// Block counters carry the call's tag in their high 32 bits: a counter whose
+// tag is not this call's is taken as 0 (fresh memory, an interrupted call),
+// and the piece that completes a block puts its counter back to 0, so the
+// next call, or the next replay of a captured graph, starts from zero.
+struct SplitWs {
+    unsigned long long *ctr;  // [nblocks]
+    float *part;              // [gridDim.x + nblocks][32 rows][64 columns]
+    unsigned long long tag;   // nonzero, < 2^32
+};
+
+__device__ __forceinline__ void store_out(const ProjParams &p, int region, int col0, int b, int c, float v) {
+    const __nv_bfloat16 o = __float2bfloat16_rn(v);
+    const int n = col0 + c;
+    if (region == 0) {
+        if (!index_ok(n < p.out_ld, p.status)) return;
+        p.q_out[(size_t)b * p.out_ld + n] = o;
+    } else {
+        const int T = p.seqlens[b];
+        if (T < 0 || T >= p.T_cap) {
+            if (c == 0 && col0 == 0) set_status(p.status, STATUS_SEQLEN);  // full cache: no append
+            return;
+        }
+        const int g = n / p.d_h, dim = n - g * p.d_h;
+        if (!index_ok(g < p.G, p.status)) return;
+        __nv_bfloat16 *cache = region == 1 ? p.k_cache : p.v_cache;
+        cache[(((size_t)b * p.G + g) * p.T_cap + T) * p.d_h + dim] = o;
+    }
+}
+
+constexpr int kStagesS = 9;
+
+template <int RB>
+__global__ void __launch_bounds__(kThreadsP, 1)
+    proj_split_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmh,
+                      const ProjParams p, const SplitWs ws) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + kStagesS * kStageB);
+    uint64_t *empty = full + kStagesS;
+    int *abort_flag = reinterpret_cast<int *>(empty + kStagesS);
+    int *last_flag = abort_flag + 1;
+    volatile int *vabort = abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int KT = p.d / kKT;
+    const int NB = p.nq + 2 * p.nk;
+    const long long U = (long long)NB * KT, C = gridDim.x;
+    const int u_begin = (int)((long long)blockIdx.x * U / C);
+    const int u_end = (int)((long long)(blockIdx.x + 1) * U / C);
+    // the CTA whose share holds unit u
+    auto cta_of = [&](long long u) { return (int)(((u + 1) * C - 1) / U); };
+    auto region_of = [&](int cb) { return cb < p.nq ? 0 : (cb < p.nq + p.nk ? 1 : 2); };
+    auto col0_of = [&](int cb) {
+        const int r = region_of(cb);
+        return (cb - (r == 0 ? 0 : (r == 1 ? p.nq : p.nq + p.nk))) * kNT;
+    };
+
+    if (tid == 0) {
+        for (int s = 0; s < kStagesS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kCW);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_wait_primary();  // h, seqlens and the workspace of the call before are settled
+
+    if (warp == kCW) {  // ---------------- TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmq);
+            tma_prefetch_desc(&tmh);
+            if (p.nk > 0) {
+                tma_prefetch_desc(&tmk);
+                tma_prefetch_desc(&tmv);
+            }
+            const uint64_t pol = l2_policy_evict_first();
+            const uint64_t pol_h = l2_policy_evict_last();  // h is read by every CTA
+            int issued = 0;
+            for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
+                const int s = it % kStagesS;
+                const uint32_t ph = (it / kStagesS) & 1;
+                if (*vabort || !mbar_wait(&empty[s], ph ^ 1, p.timeout_ns)) {
+                    set_status(p.status, STATUS_TIMEOUT);
+                    *vabort = 1;
+                    break;
+                }
+                const int cb = u / KT, kt = u - cb * KT;
+                const int region = region_of(cb);
+                const CUtensorMap *tm = region == 0 ? &tmq : (region == 1 ? &tmk : &tmv);
+                uint8_t *st = sm + s * kStageB;
+                mbar_arrive_expect_tx(&full[s], kStageB);
+                tma_load_2d(st, tm, &full[s], col0_of(cb), kt * kKT, pol);
+                tma_load_2d(st + kTileB, &tmh, &full[s], kt * kKT, p.b0, pol_h);
+                tma_load_2d(st + kTileB + kHHalf, &tmh, &full[s], kt * kKT + 64, p.b0, pol_h);
+                issued = it + 1;
+            }
+            if (*vabort)  // let copies still in flight land before the CTA exits
+                for (int it = max(0, issued - kStagesS); it < issued; ++it)
+                    mbar_wait(&full[it % kStagesS], (it / kStagesS) & 1, p.timeout_ns);
+        }
+        return;
+    }
+
+    // ---------------- MMA warps: warp w owns columns [16w, 16w + 16) of every block
+    const int g8 = lane >> 2, q4 = lane & 3;
+    float acc[RB][2][4];
+    auto zero_acc = [&]() {
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) acc[rb][nt][0] = acc[rb][nt][1] = acc[rb][nt][2] = acc[rb][nt][3] = 0.f;
+    };
+    zero_acc();
+    bool dead = false;
+    int piece_first = u_begin;  // first unit of the current piece
+    for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
+        const int s = it % kStagesS;
+        const uint32_t ph = (it / kStagesS) & 1;
+        if (!dead && (*vabort || !mbar_wait(&full[s], ph, p.timeout_ns))) {
+            dead = true;
+            *vabort = 1;
+            set_status(p.status, STATUS_TIMEOUT);
+        }
+        if (!dead) {
+            const uint32_t base = smem_u32(sm + s * kStageB);
+            const uint32_t hbase = base + kTileB;
+#pragma unroll
+            for (int ks = 0; ks < kKT / 16; ++ks) {
+                uint32_t a[RB][4];
+                const int kc = ks * 16 + ((lane >> 4) << 3);
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    const int hr = rb * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+                    ldsm_x4(hbase + (kc >> 6) * kHHalf + swz64(hr, kc & 63), a[rb][0], a[rb][1], a[rb][2],
+                            a[rb][3]);
+                }
+                const int row = ks * 16 + (((lane >> 3) & 1) << 3) + (lane & 7);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(base + swz64(row, warp * 16 + ((lane >> 4) << 3)), b0, b1, b2, b3);
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    mma_16816(acc[rb][0], a[rb], b0, b1);
+                    mma_16816(acc[rb][1], a[rb], b2, b3);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+
+        const int cb = u / KT;
+        const bool piece_end = (u + 1 == u_end) || ((u + 1) % KT == 0);
+        if (!piece_end) continue;
+        // ---------------- piece done: units [piece_first, u] of block cb
+        const int region = region_of(cb), col0 = col0_of(cb);
+        const long long blk0 = (long long)cb * KT;
+        const int c_first = cta_of(blk0), c_last = cta_of(blk0 + KT - 1);
+        if (c_first == c_last) {  // the whole block: round and store
+            if (!dead)
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int r = rb * 16 + g8 + (e >> 1) * 8, b = p.b0 + r;
+                            if (b < p.B) store_out(p, region, col0, b, warp * 16 + nt * 8 + 2 * q4 + (e & 1), acc[rb][nt][e]);
+                        }
+        } else {
+            // partial sums to this piece's slot, then count the piece on the block
+            const long long slot = (long long)blockIdx.x + cb;
+            float *mine = ws.part + slot * (32 * kNT);
+            if (!dead)
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int c = warp * 16 + nt * 8 + 2 * q4;
+                        *reinterpret_cast<float2 *>(mine + (rb * 16 + g8) * kNT + c) =
+                            make_float2(acc[rb][nt][0], acc[rb][nt][1]);
+                        *reinterpret_cast<float2 *>(mine + (rb * 16 + g8 + 8) * kNT + c) =
+                            make_float2(acc[rb][nt][2], acc[rb][nt][3]);
+                    }
+            __threadfence();
+            asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
+            if (tid == 0) {
+                int last = 0;
+                if (!*vabort) {
+                    unsigned long long *ctr = ws.ctr + cb;
+                    unsigned long long v = *reinterpret_cast<volatile unsigned long long *>(ctr);
+                    const unsigned long long n_pieces = (unsigned long long)(c_last - c_first + 1);
+                    for (int tries = 0; tries < 256; ++tries) {  // a few pieces per block contend
+                        const unsigned long long nv = (v >> 32) == ws.tag ? v + 1 : ((ws.tag << 32) | 1ull);
+                        const unsigned long long old = atomicCAS(ctr, v, nv);
+                        if (old == v) {
+                            last = (nv & 0xffffffffull) == n_pieces;
+                            break;
+                        }
+                        v = old;
+                    }
+                    if (last) {
+                        __threadfence();
+                        *ctr = 0ull;  // ready for the next call
+                    }
+                }
+                *last_flag = last;
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
+            if (*last_flag && !dead) {
+                // every piece of the block, in slot order, one rounding
+                __threadfence();
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int r = rb * 16 + g8 + hf * 8, c = warp * 16 + nt * 8 + 2 * q4;
+                            float2 sum = make_float2(0.f, 0.f);
+                            for (int cc = c_first; cc <= c_last; ++cc) {
+                                const float2 t = __ldcg(reinterpret_cast<const float2 *>(
+                                    ws.part + ((long long)cc + cb) * (32 * kNT) + r * kNT + c));
+                                sum.x += t.x;
+                                sum.y += t.y;
+                            }
+                            const int b = p.b0 + r;
+                            if (b < p.B) {
+                                store_out(p, region, col0, b, c, sum.x);
+                                store_out(p, region, col0, b, c + 1, sum.y);
+                            }
+                        }
+            }
+        }
+        zero_acc();
+        piece_first = u + 1;
+    }
+    (void)piece_first;
+    if (blockIdx.x == 0 && p.nk > 0 && p.seqlens_out)
+        for (int b = p.b0 + tid; b < min(p.B, p.b0 + RB * 16); b += kCW * 32) {
+            const int T = p.seqlens[b];
+            p.seqlens_out[b] = (T >= 0 && T < p.T_cap) ? T + 1 : T;
+        }
+}
+
 template <int RB>
 struct ProjTag {};
 
@@ -243,7 +504,71 @@ cudaError_t run_proj(const ProjParams &p, const CUtensorMap *tq, const CUtensorM
     return cudaLaunchKernelEx(&cfg, qkv_append_kernel<RB>, *tq, *tk, *tv, *th, p);
 }
 
+template <int RB>
+struct SplitTag {};
+
+// CTAs of the split-K grid: one per SM, at most one per unit.
+int split_ctas(int nblocks, int d, int num_sms) {
+    const long long units = (long long)nblocks * (d / kKT);
+    return (int)(units < num_sms ? units : num_sms);
+}
+
+template <int RB>
+cudaError_t run_split(const ProjParams &p, const SplitWs &ws, int ctas, const CUtensorMap *tq, const CUtensorMap *tk,
+                      const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t st) {
+    const size_t smem = 1024 + (size_t)kStagesS * kStageB + 2 * kStagesS * 8 + 16;
+    cudaError_t e = once_per_device<SplitTag<RB>>([&] {
+        return cudaFuncSetAttribute(proj_split_kernel<RB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(kThreadsP);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];  // programmatic dependent: the prologue may overlap the previous kernel
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, proj_split_kernel<RB>, *tq, *tk, *tv, *th, p, ws);
+}
+
+// Launches one grid per 32 sequences: the column-block kernel, or with a
+// workspace the split-K kernel.
+cudaError_t launch_proj(ProjParams p, void *workspace, int num_sms, unsigned long long tag, const CUtensorMap *tq,
+                        const CUtensorMap *tk, const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t st) {
+    const int nblocks = p.nq + 2 * p.nk;
+    SplitWs ws = {};
+    int ctas = 0;
+    if (workspace) {
+        ctas = split_ctas(nblocks, p.d, num_sms);
+        uint8_t *w = static_cast<uint8_t *>(workspace);
+        ws.ctr = reinterpret_cast<unsigned long long *>(w);
+        ws.part = reinterpret_cast<float *>(w + (((size_t)nblocks * 8 + 255) & ~size_t(255)));
+        ws.tag = tag;
+    }
+    for (int b0 = 0; b0 < p.B; b0 += 32) {  // 32 sequences per launch
+        p.b0 = b0;
+        const bool two = p.B - b0 > 16;
+        cudaError_t e;
+        if (workspace)
+            e = two ? run_split<2>(p, ws, ctas, tq, tk, tv, th, st) : run_split<1>(p, ws, ctas, tq, tk, tv, th, st);
+        else
+            e = two ? run_proj<2>(p, tq, tk, tv, th, st) : run_proj<1>(p, tq, tk, tv, th, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace
+
+size_t proj_workspace_bytes(int ncols, int d, int num_sms) {
+    if (ncols <= 0 || d <= 0 || ncols % kNT != 0 || d % kKT != 0) return 0;
+    const int nblocks = ncols / kNT;
+    const int ctas = split_ctas(nblocks, d, num_sms);
+    return (((size_t)nblocks * 8 + 255) & ~size_t(255)) + ((size_t)ctas + nblocks) * 32 * kNT * sizeof(float);
+}
 
 cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUtensorMap *tk,
                               const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t st) {
@@ -265,19 +590,13 @@ cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUt
     p.nk = a.G * a.d_h / kNT;
     p.out_ld = a.H * a.d_h;
     p.timeout_ns = a.timeout_ns;
-    for (int b0 = 0; b0 < a.B; b0 += 32) {  // 32 sequences per launch
-        p.b0 = b0;
-        const cudaError_t e =
-            (a.B - b0 > 16) ? run_proj<2>(p, tq, tk, tv, th, st) : run_proj<1>(p, tq, tk, tv, th, st);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+    return launch_proj(p, a.workspace, a.num_sms, a.tag, tq, tk, tv, th, st);
 }
 
-// out[B, N] = x[B, K] W[K, N]: the same kernel with one weight and no cache.
+// out[B, N] = x[B, K] W[K, N]: the same kernels with one weight and no cache.
 cudaError_t launch_out_project(const void *x, void *out, int B, int K, int N, unsigned *status,
-                               uint64_t timeout_ns, const CUtensorMap *tw, const CUtensorMap *tx,
-                               cudaStream_t st) {
+                               uint64_t timeout_ns, void *workspace, int num_sms, unsigned long long tag,
+                               const CUtensorMap *tw, const CUtensorMap *tx, cudaStream_t st) {
     ProjParams p = {};
     p.h = static_cast<const __nv_bfloat16 *>(x);
     p.q_out = static_cast<__nv_bfloat16 *>(out);
@@ -288,12 +607,7 @@ cudaError_t launch_out_project(const void *x, void *out, int B, int K, int N, un
     p.nk = 0;
     p.out_ld = N;
     p.timeout_ns = timeout_ns;
-    for (int b0 = 0; b0 < B; b0 += 32) {
-        p.b0 = b0;
-        const cudaError_t e = (B - b0 > 16) ? run_proj<2>(p, tw, tw, tw, tx, st) : run_proj<1>(p, tw, tw, tw, tx, st);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+    return launch_proj(p, workspace, num_sms, tag, tw, tw, tw, tx, st);
 }
 
 }  // namespace gqa

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
         lib = ctypes.CDLL(os.path.join(pkg, so))
         for name in declared_functions():
             assert hasattr(lib, name), (so, name)
-        assert lib.gqa_version() == 100
+        assert lib.gqa_version() == 101
 
 
 def test_kv_cache_bytes_matches_oracle_and_pages():

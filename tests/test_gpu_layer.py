@@ -24,11 +24,15 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("B,K,N", [(1, 128, 64), (16, 4096, 4096), (33, 256, 192), (20, 512, 640)])
-def test_out_project(gqa, B, K, N):
+@pytest.mark.parametrize("split", [False, True], ids=["column_blocks", "split_k"])
+def test_out_project(gqa, B, K, N, split):
     gen = torch.Generator().manual_seed(B + K + N)
     x = torch.randn(B, K, generator=gen).to(torch.bfloat16)
     W = (torch.randn(K, N, generator=gen) * K ** -0.5).to(torch.bfloat16)
-    out = gqa.out_project(x.cuda(), W.cuda())
+    ws = None
+    if split:
+        ws = torch.empty(gqa.project_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
+    out = gqa.out_project(x.cuda(), W.cuda(), workspace=ws)
     gqa.get_status()
     assert_close(out.cpu(), oracle.project(x, W), torch.bfloat16)
 

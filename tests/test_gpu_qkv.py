@@ -15,10 +15,15 @@ from parity import assert_close
 pytestmark = pytest.mark.gpu
 
 
-def run_and_check(gqa, x, expect_full=False):
+def _workspace(gqa, x):
+    n = gqa.project_workspace_bytes((x.H + 2 * x.G) * x.d_h, x.d)
+    return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+def run_and_check(gqa, x, expect_full=False, split=False):
     kc, vc = x.k_cache.cuda(), x.v_cache.cuda()
     q, sl_out = gqa.qkv_append(x.h.cuda(), x.W_Q.cuda(), x.W_K.cuda(), x.W_V.cuda(), kc, vc,
-                               x.seqlens.cuda())
+                               x.seqlens.cuda(), workspace=_workspace(gqa, x) if split else None)
     if expect_full:
         with pytest.raises(gqa.GQAError) as ei:
             gqa.get_status()
@@ -48,20 +53,57 @@ def run_and_check(gqa, x, expect_full=False):
     (33, 256, 8, 8, 64, 10, [i % 10 for i in range(33)]),   # two launches, G = H (MHA)
     (5, 128, 32, 1, 128, 4, [3, 0, 1, 2, 3]),                # MQA
 ])
-def test_qkv_append_small(gqa, B, d, H, G, d_h, T, seqlens):
+@pytest.mark.parametrize("split", [False, True], ids=["column_blocks", "split_k"])
+def test_qkv_append_small(gqa, B, d, H, G, d_h, T, seqlens, split):
     x = gi.qkv_inputs(B, d, H, G, d_h, T, seed=B + d, seqlens=seqlens)
-    run_and_check(gqa, x)
+    run_and_check(gqa, x, split=split)
 
 
-def test_qkv_append_full_cache_is_not_written(gqa):
+@pytest.mark.parametrize("split", [False, True], ids=["column_blocks", "split_k"])
+def test_qkv_append_full_cache_is_not_written(gqa, split):
     x = gi.qkv_inputs(4, 256, 8, 2, 64, 6, seed=3, seqlens=[6, 2, 6, 5])
-    run_and_check(gqa, x, expect_full=True)
+    run_and_check(gqa, x, expect_full=True, split=split)
 
 
-def test_qkv_append_llama2_7b_full(gqa):
+@pytest.mark.parametrize("split", [False, True], ids=["column_blocks", "split_k"])
+def test_qkv_append_llama2_7b_full(gqa, split):
     """B=16, d=4096, H=32, G=8, d_h=128, T_cap=4096 (last free slot)."""
     x = gi.workload_inputs("qkv_append_llama2_7b")
-    run_and_check(gqa, x)
+    run_and_check(gqa, x, split=split)
+
+
+def test_split_k_is_deterministic_and_graph_replayable(gqa):
+    """The split-K kernel adds a block's partial sums in slot order whichever CTA
+    finishes last, and resets the block counters for the next call: repeated
+    calls, and one call captured in a CUDA graph and replayed with h changed in
+    place, give the bits of eager calls."""
+    x = gi.qkv_inputs(16, 4096, 32, 8, 128, 8, seed=21, seqlens=[3] * 16)
+    h, wq, wk, wv = x.h.cuda(), x.W_Q.cuda(), x.W_K.cuda(), x.W_V.cuda()
+    kc, vc, sl = x.k_cache.cuda(), x.v_cache.cuda(), x.seqlens.cuda()
+    ws = _workspace(gqa, x)
+    q = torch.empty((16, 32, 128), dtype=torch.bfloat16, device="cuda")
+    sl_out = torch.empty_like(sl)
+    ref = [gqa.qkv_append(h, wq, wk, wv, kc, vc, sl, workspace=ws)[0].clone() for _ in range(3)]
+    assert torch.equal(ref[0], ref[1]) and torch.equal(ref[0], ref[2])
+    gqa.qkv_append(h, wq, wk, wv, kc, vc, sl, q_out=q, seqlens_out=sl_out, workspace=ws)
+    torch.cuda.synchronize()
+    graph, s = torch.cuda.CUDAGraph(), torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=s):
+        gqa.qkv_append(h, wq, wk, wv, kc, vc, sl, q_out=q, seqlens_out=sl_out, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    gen = torch.Generator().manual_seed(22)
+    for i in range(4):
+        h.copy_(torch.randn(h.shape, generator=gen).to(torch.bfloat16))
+        graph.replay()
+        got = q.clone()
+        eager = gqa.qkv_append(h, wq, wk, wv, kc.clone(), vc.clone(), sl)[0]  # column-block kernel
+        eager_split = gqa.qkv_append(h, wq, wk, wv, kc.clone(), vc.clone(), sl,
+                                     workspace=_workspace(gqa, x))[0]
+        torch.cuda.synchronize()
+        gqa.get_status()
+        assert torch.equal(got, eager_split), "replay %d" % i
+        assert_close(got.cpu(), eager.cpu().double(), torch.bfloat16)
 
 
 def test_qkv_then_decode_sees_the_new_token(gqa):
