@@ -289,6 +289,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const bool split_p = seq_len <= kSplitPMaxLen;
                 uint32_t pl[4] = {0u, 0u, 0u, 0u};
                 if (split_p) {
+                    // the row sum takes the same P_hi + P_lo the products use, so that
+                    // numerator and denominator agree (with P_hi alone it would be off
+                    // by the rounding of P, ~2^-9 relative on short sequences)
+                    float ls_a = 0.f, ls_b = 0.f;
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
                         const float2 ha = unpack_bf16x2(pa[2 * nt + 0]);
@@ -297,7 +301,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                                                      fast_exp2(sc[nt][1] - mu_a) - ha.y);
                         pl[2 * nt + 1] = pack_bf16x2(fast_exp2(sc[nt][2] - mu_b) - hb.x,
                                                      fast_exp2(sc[nt][3] - mu_b) - hb.y);
+                        const float2 la = unpack_bf16x2(pl[2 * nt + 0]);
+                        const float2 lb = unpack_bf16x2(pl[2 * nt + 1]);
+                        ls_a += la.x + la.y;
+                        ls_b += lb.x + lb.y;
                     }
+                    l_a += ls_a;
+                    l_b += ls_b;
                 }
                 {
                     const int tok = row0 + (((lane >> 3) & 1) << 3) + (lane & 7);

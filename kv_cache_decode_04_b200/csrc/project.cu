@@ -222,25 +222,32 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 // Split-K variant for every SM.  The column-block kernel above gives each
 // 64-column block of the weights one CTA, which leaves SMs idle whenever
 // there are fewer blocks than SMs (96 for the Llama-2-7B Q/K/V projection, 64
-// for its W_O).  Here the units (column block cb, 128-row K tile kt), cb-major,
-// are laid end to end and cut into gridDim.x equal shares, one CTA per SM.  A
-// share's part of one block is a piece, with slot c + cb (distinct for all
-// pieces, as for the decode records).  A piece that covers its whole block is
-// rounded and stored directly; any other writes its fp32 partial sums to its
-// slot in the workspace and counts itself on the block's counter, and the
-// piece that completes the count adds the block's partials up in slot order
-// (the same order whichever piece finishes last: deterministic), rounds once
-// and stores.  Each MMA warp owns 16 of the block's 64 columns over all K
-// steps, so a warp's partial needs no reduction across warps.
+// for its W_O).  Here each block's 128-row K tiles are also cut into ks equal
+// row ranges: items (block cb, range s), item = s * nblocks + cb, taken by
+// CTA item mod gridDim.x (one CTA per SM) in increasing order.  ks is chosen
+// on the host to minimise the largest CTA's tile count.  Items of the same
+// range start together on different CTAs, so the CTAs running at one time
+// read the same weight rows (different column blocks): the DRAM pages a row
+// spans are read by many CTAs at once, as in the column-block kernel.  (Equal
+// shares of a block-major line were tried first: concurrent CTAs then sat on
+// different rows, and the kernel ran at half the column-block kernel's rate.)
+// With ks = 1 an item is a whole block, rounded and stored directly;
+// otherwise each item writes its fp32 partial sums to slot `item` of the
+// workspace and counts itself on the block's counter, and the item that
+// completes the count adds the block's ks partials in range order (the same
+// order whichever finishes last: deterministic), rounds once and stores.
+// Each MMA warp owns 16 of the block's 64 columns over all K steps, so a
+// warp's partial needs no reduction across warps.
 //
 // Block counters carry the call's tag in their high 32 bits: a counter whose
 // tag is not this call's is taken as 0 (fresh memory, an interrupted call),
-// and the piece that completes a block puts its counter back to 0, so the
+// and the item that completes a block puts its counter back to 0, so the
 // next call, or the next replay of a captured graph, starts from zero.
 struct SplitWs {
     unsigned long long *ctr;  // [nblocks]
-    float *part;              // [gridDim.x + nblocks][32 rows][64 columns]
+    float *part;              // [ks * nblocks][32 rows][64 columns]
     unsigned long long tag;   // nonzero, < 2^32
+    int ks;                   // row ranges per block
 };
 
 __device__ __forceinline__ void store_out(const ProjParams &p, int region, int col0, int b, int c, float v) {
@@ -281,16 +288,14 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int KT = p.d / kKT;
     const int NB = p.nq + 2 * p.nk;
-    const long long U = (long long)NB * KT, C = gridDim.x;
-    const int u_begin = (int)((long long)blockIdx.x * U / C);
-    const int u_end = (int)((long long)(blockIdx.x + 1) * U / C);
-    // the CTA whose share holds unit u
-    auto cta_of = [&](long long u) { return (int)(((u + 1) * C - 1) / U); };
+    const int n_items = NB * ws.ks;
     auto region_of = [&](int cb) { return cb < p.nq ? 0 : (cb < p.nq + p.nk ? 1 : 2); };
     auto col0_of = [&](int cb) {
         const int r = region_of(cb);
         return (cb - (r == 0 ? 0 : (r == 1 ? p.nq : p.nq + p.nk))) * kNT;
     };
+    // K tiles [kt_lo(r), kt_lo(r + 1)) of row range r
+    auto kt_lo = [&](int r) { return (int)((long long)r * KT / ws.ks); };
 
     if (tid == 0) {
         for (int s = 0; s < kStagesS; ++s) {
@@ -313,24 +318,26 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             }
             const uint64_t pol = l2_policy_evict_first();
             const uint64_t pol_h = l2_policy_evict_last();  // h is read by every CTA
-            int issued = 0;
-            for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
-                const int s = it % kStagesS;
-                const uint32_t ph = (it / kStagesS) & 1;
-                if (*vabort || !mbar_wait(&empty[s], ph ^ 1, p.timeout_ns)) {
-                    set_status(p.status, STATUS_TIMEOUT);
-                    *vabort = 1;
-                    break;
-                }
-                const int cb = u / KT, kt = u - cb * KT;
-                const int region = region_of(cb);
+            int issued = 0, it = 0;
+            for (int item = blockIdx.x; item < n_items && !*vabort; item += gridDim.x) {
+                const int cb = item % NB, rg = item / NB;
+                const int region = region_of(cb), col0 = col0_of(cb);
                 const CUtensorMap *tm = region == 0 ? &tmq : (region == 1 ? &tmk : &tmv);
-                uint8_t *st = sm + s * kStageB;
-                mbar_arrive_expect_tx(&full[s], kStageB);
-                tma_load_2d(st, tm, &full[s], col0_of(cb), kt * kKT, pol);
-                tma_load_2d(st + kTileB, &tmh, &full[s], kt * kKT, p.b0, pol_h);
-                tma_load_2d(st + kTileB + kHHalf, &tmh, &full[s], kt * kKT + 64, p.b0, pol_h);
-                issued = it + 1;
+                for (int kt = kt_lo(rg); kt < kt_lo(rg + 1); ++kt, ++it) {
+                    const int s = it % kStagesS;
+                    const uint32_t ph = (it / kStagesS) & 1;
+                    if (*vabort || !mbar_wait(&empty[s], ph ^ 1, p.timeout_ns)) {
+                        set_status(p.status, STATUS_TIMEOUT);
+                        *vabort = 1;
+                        break;
+                    }
+                    uint8_t *st = sm + s * kStageB;
+                    mbar_arrive_expect_tx(&full[s], kStageB);
+                    tma_load_2d(st, tm, &full[s], col0, kt * kKT, pol);
+                    tma_load_2d(st + kTileB, &tmh, &full[s], kt * kKT, p.b0, pol_h);
+                    tma_load_2d(st + kTileB + kHHalf, &tmh, &full[s], kt * kKT + 64, p.b0, pol_h);
+                    issued = it + 1;
+                }
             }
             if (*vabort)  // let copies still in flight land before the CTA exits
                 for (int it = max(0, issued - kStagesS); it < issued; ++it)
@@ -350,8 +357,10 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     };
     zero_acc();
     bool dead = false;
-    int piece_first = u_begin;  // first unit of the current piece
-    for (int u = u_begin, it = 0; u < u_end; ++u, ++it) {
+    int it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const int cb = item % NB, rg = item / NB;
+      for (int kt = kt_lo(rg); kt < kt_lo(rg + 1); ++kt, ++it) {
         const int s = it % kStagesS;
         const uint32_t ph = (it / kStagesS) & 1;
         if (!dead && (*vabort || !mbar_wait(&full[s], ph, p.timeout_ns))) {
@@ -384,15 +393,10 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
-
-        const int cb = u / KT;
-        const bool piece_end = (u + 1 == u_end) || ((u + 1) % KT == 0);
-        if (!piece_end) continue;
-        // ---------------- piece done: units [piece_first, u] of block cb
+      }
+        // ---------------- item done: rows [kt_lo(rg), kt_lo(rg + 1)) of block cb
         const int region = region_of(cb), col0 = col0_of(cb);
-        const long long blk0 = (long long)cb * KT;
-        const int c_first = cta_of(blk0), c_last = cta_of(blk0 + KT - 1);
-        if (c_first == c_last) {  // the whole block: round and store
+        if (ws.ks == 1) {  // the whole block: round and store
             if (!dead)
 #pragma unroll
                 for (int rb = 0; rb < RB; ++rb)
@@ -404,9 +408,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                             if (b < p.B) store_out(p, region, col0, b, warp * 16 + nt * 8 + 2 * q4 + (e & 1), acc[rb][nt][e]);
                         }
         } else {
-            // partial sums to this piece's slot, then count the piece on the block
-            const long long slot = (long long)blockIdx.x + cb;
-            float *mine = ws.part + slot * (32 * kNT);
+            // partial sums to this item's slot, then count the item on the block
+            float *mine = ws.part + (long long)item * (32 * kNT);
             if (!dead)
 #pragma unroll
                 for (int rb = 0; rb < RB; ++rb)
@@ -425,12 +428,11 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 if (!*vabort) {
                     unsigned long long *ctr = ws.ctr + cb;
                     unsigned long long v = *reinterpret_cast<volatile unsigned long long *>(ctr);
-                    const unsigned long long n_pieces = (unsigned long long)(c_last - c_first + 1);
-                    for (int tries = 0; tries < 256; ++tries) {  // a few pieces per block contend
+                    for (int tries = 0; tries < 256; ++tries) {  // ks items per block contend
                         const unsigned long long nv = (v >> 32) == ws.tag ? v + 1 : ((ws.tag << 32) | 1ull);
                         const unsigned long long old = atomicCAS(ctr, v, nv);
                         if (old == v) {
-                            last = (nv & 0xffffffffull) == n_pieces;
+                            last = (nv & 0xffffffffull) == (unsigned long long)ws.ks;
                             break;
                         }
                         v = old;
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             }
             asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
             if (*last_flag && !dead) {
-                // every piece of the block, in slot order, one rounding
+                // the block's ks partials, in range order, one rounding
                 __threadfence();
 #pragma unroll
                 for (int rb = 0; rb < RB; ++rb)
@@ -454,9 +456,9 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                         for (int hf = 0; hf < 2; ++hf) {
                             const int r = rb * 16 + g8 + hf * 8, c = warp * 16 + nt * 8 + 2 * q4;
                             float2 sum = make_float2(0.f, 0.f);
-                            for (int cc = c_first; cc <= c_last; ++cc) {
+                            for (int r2 = 0; r2 < ws.ks; ++r2) {
                                 const float2 t = __ldcg(reinterpret_cast<const float2 *>(
-                                    ws.part + ((long long)cc + cb) * (32 * kNT) + r * kNT + c));
+                                    ws.part + ((long long)r2 * NB + cb) * (32 * kNT) + r * kNT + c));
                                 sum.x += t.x;
                                 sum.y += t.y;
                             }
@@ -469,9 +471,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             }
         }
         zero_acc();
-        piece_first = u + 1;
     }
-    (void)piece_first;
+
     if (blockIdx.x == 0 && p.nk > 0 && p.seqlens_out)
         for (int b = p.b0 + tid; b < min(p.B, p.b0 + RB * 16); b += kCW * 32) {
             const int T = p.seqlens[b];
@@ -507,10 +508,33 @@ cudaError_t run_proj(const ProjParams &p, const CUtensorMap *tq, const CUtensorM
 template <int RB>
 struct SplitTag {};
 
-// CTAs of the split-K grid: one per SM, at most one per unit.
-int split_ctas(int nblocks, int d, int num_sms) {
-    const long long units = (long long)nblocks * (d / kKT);
-    return (int)(units < num_sms ? units : num_sms);
+// Row ranges per block (ks) and CTAs of the split-K grid.  The busiest CTA
+// streams ceil(nblocks * ks / CTAs) * ceil(KT / ks) tiles; ks is the smallest
+// split within 15 % of the fewest such tiles (more ranges cost partial-sum
+// traffic and reductions for little gain).  One CTA per SM, at most one per
+// item.
+struct SplitPlan {
+    int ks, ctas;
+};
+SplitPlan split_plan(int nblocks, int d, int num_sms) {
+    const int KT = d / kKT;
+    auto cost = [&](int ks) {
+        const long long items = (long long)nblocks * ks;
+        const long long ctas = items < num_sms ? items : num_sms;
+        return ((items + ctas - 1) / ctas) * ((KT + ks - 1) / ks);
+    };
+    long long best = -1;
+    for (int ks = 1; ks <= KT; ++ks)
+        if (best < 0 || cost(ks) < best) best = cost(ks);
+    SplitPlan plan = {1, 1};
+    for (int ks = 1; ks <= KT; ++ks)
+        if (cost(ks) * 100 <= best * 115) {
+            const long long items = (long long)nblocks * ks;
+            plan.ks = ks;
+            plan.ctas = (int)(items < num_sms ? items : num_sms);
+            break;
+        }
+    return plan;
 }
 
 template <int RB>
@@ -542,11 +566,13 @@ cudaError_t launch_proj(ProjParams p, void *workspace, int num_sms, unsigned lon
     SplitWs ws = {};
     int ctas = 0;
     if (workspace) {
-        ctas = split_ctas(nblocks, p.d, num_sms);
+        const SplitPlan plan = split_plan(nblocks, p.d, num_sms);
+        ctas = plan.ctas;
         uint8_t *w = static_cast<uint8_t *>(workspace);
         ws.ctr = reinterpret_cast<unsigned long long *>(w);
         ws.part = reinterpret_cast<float *>(w + (((size_t)nblocks * 8 + 255) & ~size_t(255)));
         ws.tag = tag;
+        ws.ks = plan.ks;
     }
     for (int b0 = 0; b0 < p.B; b0 += 32) {  // 32 sequences per launch
         p.b0 = b0;
@@ -566,8 +592,8 @@ cudaError_t launch_proj(ProjParams p, void *workspace, int num_sms, unsigned lon
 size_t proj_workspace_bytes(int ncols, int d, int num_sms) {
     if (ncols <= 0 || d <= 0 || ncols % kNT != 0 || d % kKT != 0) return 0;
     const int nblocks = ncols / kNT;
-    const int ctas = split_ctas(nblocks, d, num_sms);
-    return (((size_t)nblocks * 8 + 255) & ~size_t(255)) + ((size_t)ctas + nblocks) * 32 * kNT * sizeof(float);
+    const SplitPlan plan = split_plan(nblocks, d, num_sms);
+    return (((size_t)nblocks * 8 + 255) & ~size_t(255)) + (size_t)plan.ks * nblocks * 32 * kNT * sizeof(float);
 }
 
 cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUtensorMap *tk,

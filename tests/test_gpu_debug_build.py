@@ -40,7 +40,9 @@ SUBSET = [
 
 
 def _child(args, extra_env, timeout=900):
-    env = dict(os.environ, GQA_LIB="debug", **extra_env)
+    env = dict(os.environ)
+    env["GQA_LIB"] = "debug"
+    env.update(extra_env)
     return subprocess.run([sys.executable, *args], cwd=ROOT, env=env, capture_output=True, text=True,
                           timeout=timeout)
 
