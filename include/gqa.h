@@ -248,14 +248,15 @@ GQA_API int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *
  *   workspace         device, >= gqa_project_workspace_bytes((H + 2G) d_h, d)
  *                     bytes, 256-byte aligned, or NULL (see below)
  *   Supported: dt = GQA_BF16, d a multiple of 128, d_h in {64, 128}.
- * Internally: a skinny GEMM bound by reading the weights once.  Without a
- * workspace, one CTA per 64 output columns; with one, the (column block,
- * 128-row K tile) units are cut into equal shares, one CTA per SM, and the
- * blocks split between CTAs are added up in a fixed order from fp32 partial
- * sums in the workspace (same results on every call; they may differ from
- * the workspace-free kernel's in the last bit, since the sums are grouped
- * differently).  The workspace needs no initialisation; calls that run
- * concurrently need separate workspaces.
+ * Internally: a skinny GEMM bound by reading the weights once, one CTA per
+ * 64 output columns.  With a workspace and fewer column blocks than half the
+ * SMs, each block's rows are also split into floor(SMs / blocks) ranges on
+ * separate CTAs, all in one wave, and the ranges' fp32 partial sums are added
+ * in a fixed order from the workspace (same results on every call; they may
+ * differ from the unsplit kernel's in the last bit, since the sums are
+ * grouped differently).  With more blocks the workspace is not used.  It
+ * needs no initialisation; calls that run concurrently need separate
+ * workspaces.
  */
 GQA_API int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V,
                            void *q_out, void *k_cache, void *v_cache, const int32_t *seqlens,

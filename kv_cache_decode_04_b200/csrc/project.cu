@@ -20,6 +20,8 @@
 // warps split each tile's sixteen-row K-steps and run warp-level bf16 MMAs (B
 // padded to 16-row blocks), then the four partial sums are added in a fixed
 // order in shared memory, rounded once to bf16 and written.
+#include <cstdlib>
+
 #include "common.cuh"
 #include "gqa.h"
 #include "internal.h"
@@ -508,33 +510,26 @@ cudaError_t run_proj(const ProjParams &p, const CUtensorMap *tq, const CUtensorM
 template <int RB>
 struct SplitTag {};
 
-// Row ranges per block (ks) and CTAs of the split-K grid.  The busiest CTA
-// streams ceil(nblocks * ks / CTAs) * ceil(KT / ks) tiles; ks is the smallest
-// split within 15 % of the fewest such tiles (more ranges cost partial-sum
-// traffic and reductions for little gain).  One CTA per SM, at most one per
-// item.
+// Row ranges per block (ks) and CTAs of the split-K grid.  Weight tiles are
+// 128-byte column segments of 128 rows; they stream at full rate only while
+// the CTAs on neighbouring column blocks move down the rows together, as the
+// column-block kernel's do.  So every item must run in the one wave:
+// ks = floor(SMs / blocks) (e.g. 2 for a 64-block W_O on 148 SMs), and with
+// ks = 1 the column-block kernel is used.  Measured on the 96-block Q/K/V
+// projection: ks = 1, 2, 3, 4 and 8 took 17.8, 24.4, 19.8, 22.2 and 33.5 us
+// against 16.5 us for the column-block kernel.
 struct SplitPlan {
     int ks, ctas;
 };
 SplitPlan split_plan(int nblocks, int d, int num_sms) {
     const int KT = d / kKT;
-    auto cost = [&](int ks) {
-        const long long items = (long long)nblocks * ks;
-        const long long ctas = items < num_sms ? items : num_sms;
-        return ((items + ctas - 1) / ctas) * ((KT + ks - 1) / ks);
-    };
-    long long best = -1;
-    for (int ks = 1; ks <= KT; ++ks)
-        if (best < 0 || cost(ks) < best) best = cost(ks);
-    SplitPlan plan = {1, 1};
-    for (int ks = 1; ks <= KT; ++ks)
-        if (cost(ks) * 100 <= best * 115) {
-            const long long items = (long long)nblocks * ks;
-            plan.ks = ks;
-            plan.ctas = (int)(items < num_sms ? items : num_sms);
-            break;
-        }
-    return plan;
+    int ks = nblocks > 0 ? num_sms / nblocks : 1;
+    // GQA_PROJ_KS=k forces k row ranges (tests of the split paths, measurements)
+    const char *force = getenv("GQA_PROJ_KS");
+    if (force && atoi(force) > 0) ks = atoi(force);
+    if (ks > KT) ks = KT;
+    if (ks < 1) ks = 1;
+    return {ks, nblocks * ks};
 }
 
 template <int RB>
@@ -574,6 +569,7 @@ cudaError_t launch_proj(ProjParams p, void *workspace, int num_sms, unsigned lon
         ws.tag = tag;
         ws.ks = plan.ks;
     }
+    if (workspace && ws.ks == 1 && !getenv("GQA_PROJ_KS")) workspace = nullptr;  // nothing to split
     for (int b0 = 0; b0 < p.B; b0 += 32) {  // 32 sequences per launch
         p.b0 = b0;
         const bool two = p.B - b0 > 16;

@@ -77,11 +77,12 @@ def test_split_k_is_deterministic_and_graph_replayable(gqa):
     finishes last, and resets the block counters for the next call: repeated
     calls, and one call captured in a CUDA graph and replayed with h changed in
     place, give the bits of eager calls."""
-    x = gi.qkv_inputs(16, 4096, 32, 8, 128, 8, seed=21, seqlens=[3] * 16)
+    # 48 column blocks: each is split over three CTAs on a 148-SM part
+    x = gi.qkv_inputs(16, 4096, 16, 4, 128, 8, seed=21, seqlens=[3] * 16)
     h, wq, wk, wv = x.h.cuda(), x.W_Q.cuda(), x.W_K.cuda(), x.W_V.cuda()
     kc, vc, sl = x.k_cache.cuda(), x.v_cache.cuda(), x.seqlens.cuda()
     ws = _workspace(gqa, x)
-    q = torch.empty((16, 32, 128), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((16, 16, 128), dtype=torch.bfloat16, device="cuda")
     sl_out = torch.empty_like(sl)
     ref = [gqa.qkv_append(h, wq, wk, wv, kc, vc, sl, workspace=ws)[0].clone() for _ in range(3)]
     assert torch.equal(ref[0], ref[1]) and torch.equal(ref[0], ref[2])
