@@ -249,14 +249,14 @@ GQA_API int gqa_meanpool_kv(const void *WK, const void *WV, void *WK_out, void *
  *                     bytes, 256-byte aligned, or NULL (see below)
  *   Supported: dt = GQA_BF16, d a multiple of 128, d_h in {64, 128}.
  * Internally: a skinny GEMM bound by reading the weights once, one CTA per
- * 64 output columns.  With a workspace and fewer column blocks than half the
- * SMs, each block's rows are also split into floor(SMs / blocks) ranges on
- * separate CTAs, all in one wave, and the ranges' fp32 partial sums are added
- * in a fixed order from the workspace (same results on every call; they may
- * differ from the unsplit kernel's in the last bit, since the sums are
- * grouped differently).  With more blocks the workspace is not used.  It
- * needs no initialisation; calls that run concurrently need separate
- * workspaces.
+ * 64 output columns.  With a workspace and at most a quarter as many column
+ * blocks as SMs, each block's rows are also split into floor(SMs / blocks)
+ * ranges on separate CTAs, all in one wave, and the ranges' fp32 partial sums
+ * are added in a fixed order from the workspace (same results on every call;
+ * they may differ from the unsplit kernel's in the last bit, since the sums
+ * are grouped differently).  With more blocks the workspace is not used (on
+ * B200 the split measured slower there).  It needs no initialisation; calls
+ * that run concurrently need separate workspaces.
  */
 GQA_API int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V,
                            void *q_out, void *k_cache, void *v_cache, const int32_t *seqlens,
@@ -317,8 +317,8 @@ GQA_API int gqa_out_project(const void *x, const void *W, void *out, int B, int 
  * k/v appended at seqlens[b]), then gqa_decode_window over seqlens_out
  * (which includes the new token), then gqa_out_project of the attention
  * output with W_O into out [B, d].  q and the attention output are kept in
- * bf16 in the workspace between the steps; both projections use the split-K
- * kernel, with their partial sums in the workspace too.
+ * bf16 in the workspace between the steps, and so are the projections'
+ * partial sums when a projection takes the split-K kernel.
  *   W_O          device, [H*d_h, d] bf16
  *   seqlens_out  required: the lengths after the append
  *   workspace    >= gqa_layer_decode_workspace_bytes(...), 256-byte aligned

@@ -557,6 +557,30 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
     float M = -INFINITY, L = 0.f;
     const unsigned long long gen = dec::call_generation(p);
     const bool pre_ok = __all_sync(0xffffffffu, wait_flag(&p.ws_flag[0], gen, p.timeout_ns));  // tile prefix
+    if (threadIdx.x == 0) {
+        // Count this CTA as started: its read of the header is behind it.  The
+        // last CTA to count stores this call's generation for the next call (all
+        // CTAs have derived theirs by then), so the store is off the grid's tail.
+        // The count was zeroed before the prefix flag; a CTA that never saw that
+        // flag does not count itself (the grid then never completes the count)
+        // and invalidates the header.  A wait that runs out later marks the
+        // count bad and invalidates the header itself (below), so the next call
+        // starts from a fresh random generation rather than one that flags left
+        // by this call could match.
+        if (!pre_ok) {
+            p.ws_hdr[dec::HDR_CHECK] = 0ull;
+        } else {
+            const unsigned long long prev = atomicAdd(&p.ws_hdr[dec::HDR_DONE], 1ull);
+            if ((prev & 0xffffffffull) == (unsigned long long)gridDim.x - 1) {
+                if (prev >> 32) {
+                    p.ws_hdr[dec::HDR_CHECK] = 0ull;
+                } else {
+                    p.ws_hdr[dec::HDR_EPOCH] = gen;
+                    p.ws_hdr[dec::HDR_CHECK] = gen ^ dec::kHdrMagic;
+                }
+            }
+        }
+    }
     bool ok = pre_ok;
     const int *cu = p.ws_cu;
     const int ntb = ok ? (cu[b + 1] - cu[b]) / p.G : 0;
@@ -629,32 +653,14 @@ __global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, 
     __syncthreads();
     pdl_launch_dependents();  // the next decode's split kernel may start its prologue
     if (warp != 0) return;
-    if (lane == 0) {
-        // Count this CTA as finished (its read of the header is behind it).  The
-        // last CTA of the grid stores this call's generation for the next call,
-        // or, if a wait of any CTA ran out, a header that fails its check, so
-        // that the next call starts from a fresh random generation rather than
-        // one that flags left by this call could match.  The count was zeroed
-        // before the prefix flag; a CTA that never saw that flag does not count
-        // itself (the grid then never completes the count) and invalidates the
-        // header directly.
+    if (lane == 0 && pre_ok) {
         int bad = 0;
 #pragma unroll
         for (int w = 0; w < NW; ++w) bad |= red_bad[w];
-        if (bad & 2) {
-            p.ws_hdr[dec::HDR_CHECK] = 0ull;
-        } else {
+        if (bad) {  // a record wait ran out: no valid header from this call
+            atomicAdd(&p.ws_hdr[dec::HDR_DONE], 1ull << 32);
             __threadfence();
-            const unsigned long long prev = atomicAdd(&p.ws_hdr[dec::HDR_DONE], 1ull + (bad ? (1ull << 32) : 0ull));
-            if ((prev & 0xffffffffull) == (unsigned long long)gridDim.x - 1) {
-                __threadfence();
-                if (bad || (prev >> 32)) {
-                    p.ws_hdr[dec::HDR_CHECK] = 0ull;
-                } else {
-                    p.ws_hdr[dec::HDR_EPOCH] = gen;
-                    p.ws_hdr[dec::HDR_CHECK] = gen ^ dec::kHdrMagic;
-                }
-            }
+            p.ws_hdr[dec::HDR_CHECK] = 0ull;
         }
     }
     float Mt = -INFINITY;

@@ -21,6 +21,7 @@
 // padded to 16-row blocks), then the four partial sums are added in a fixed
 // order in shared memory, rounded once to bf16 and written.
 #include <cstdlib>
+#include <cstring>
 
 #include "common.cuh"
 #include "gqa.h"
@@ -226,8 +227,9 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 // there are fewer blocks than SMs (96 for the Llama-2-7B Q/K/V projection, 64
 // for its W_O).  Here each block's 128-row K tiles are also cut into ks equal
 // row ranges: items (block cb, range s), item = s * nblocks + cb, taken by
-// CTA item mod gridDim.x (one CTA per SM) in increasing order.  ks is chosen
-// on the host to minimise the largest CTA's tile count.  Items of the same
+// CTA item mod gridDim.x in increasing order.  The host takes
+// ks = floor(SMs / blocks), so every item has a CTA of its own in one wave
+// (split_plan below).  Items of the same
 // range start together on different CTAs, so the CTAs running at one time
 // read the same weight rows (different column blocks): the DRAM pages a row
 // spans are read by many CTAs at once, as in the column-block kernel.  (Equal
@@ -514,10 +516,12 @@ struct SplitTag {};
 // 128-byte column segments of 128 rows; they stream at full rate only while
 // the CTAs on neighbouring column blocks move down the rows together, as the
 // column-block kernel's do.  So every item must run in the one wave:
-// ks = floor(SMs / blocks) (e.g. 2 for a 64-block W_O on 148 SMs), and with
-// ks = 1 the column-block kernel is used.  Measured on the 96-block Q/K/V
-// projection: ks = 1, 2, 3, 4 and 8 took 17.8, 24.4, 19.8, 22.2 and 33.5 us
-// against 16.5 us for the column-block kernel.
+// ks = floor(SMs / blocks).  The split pays only when it spreads the weights
+// over several times the SMs the column-block kernel would use: graph-timed
+// with the weights cycled past L2, a 64-block W_O took 12.7 us split in two
+// (128 CTAs) against 10.1 us in column blocks, and the 96-block Q/K/V
+// projection 12.1 us against 11.7 us.  Hence kMinSplit.
+constexpr int kMinSplit = 4;
 struct SplitPlan {
     int ks, ctas;
 };
@@ -553,11 +557,24 @@ cudaError_t run_split(const ProjParams &p, const SplitWs &ws, int ctas, const CU
     return cudaLaunchKernelEx(&cfg, proj_split_kernel<RB>, *tq, *tk, *tv, *th, p, ws);
 }
 
-// Launches one grid per 32 sequences: the column-block kernel, or with a
-// workspace the split-K kernel.
+// Which kernel a projection takes: the column-block kernel, or with a
+// workspace and at most a quarter as many column blocks as SMs the split-K
+// kernel (split_plan).  GQA_PROJ_KERNEL=column|split forces one (tests of
+// both paths, A/Bs).
+enum class ProjKernel { Column, Split };
+ProjKernel proj_kernel(int nblocks, int d, int num_sms, bool have_ws) {
+    const char *force = getenv("GQA_PROJ_KERNEL");
+    if (force && !strcmp(force, "column")) return ProjKernel::Column;
+    if (force && !strcmp(force, "split")) return have_ws ? ProjKernel::Split : ProjKernel::Column;
+    return have_ws && split_plan(nblocks, d, num_sms).ks >= kMinSplit ? ProjKernel::Split : ProjKernel::Column;
+}
+
+// Launches one grid per 32 sequences.
 cudaError_t launch_proj(ProjParams p, void *workspace, int num_sms, unsigned long long tag, const CUtensorMap *tq,
                         const CUtensorMap *tk, const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t st) {
     const int nblocks = p.nq + 2 * p.nk;
+    const ProjKernel kind = proj_kernel(nblocks, p.d, num_sms, workspace != nullptr);
+    if (kind == ProjKernel::Column) workspace = nullptr;
     SplitWs ws = {};
     int ctas = 0;
     if (workspace) {
@@ -569,7 +586,6 @@ cudaError_t launch_proj(ProjParams p, void *workspace, int num_sms, unsigned lon
         ws.tag = tag;
         ws.ks = plan.ks;
     }
-    if (workspace && ws.ks == 1 && !getenv("GQA_PROJ_KS")) workspace = nullptr;  // nothing to split
     for (int b0 = 0; b0 < p.B; b0 += 32) {  // 32 sequences per launch
         p.b0 = b0;
         const bool two = p.B - b0 > 16;

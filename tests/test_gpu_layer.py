@@ -23,14 +23,22 @@ from parity import assert_close, assert_strict, errors
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,K,N", [(1, 128, 64), (16, 4096, 4096), (33, 256, 192), (20, 512, 640)])
-@pytest.mark.parametrize("split", [False, True], ids=["column_blocks", "split_k"])
-def test_out_project(gqa, B, K, N, split):
+@pytest.mark.parametrize("B,K,N", [(1, 128, 64), (16, 4096, 4096), (33, 256, 192), (20, 512, 640),
+                                   (16, 4096, 1024)])
+@pytest.mark.parametrize("kernel", ["default", "column", "split"])
+def test_out_project(gqa, monkeypatch, B, K, N, kernel):
+    """Both projection kernels (GQA_PROJ_KERNEL forces one), and the default
+    choice with a workspace: split-K for few column blocks (N = 64, 192, 640,
+    1024 on 148 SMs), column blocks for N = 4096."""
+    if kernel == "default":
+        monkeypatch.delenv("GQA_PROJ_KERNEL", raising=False)
+    else:
+        monkeypatch.setenv("GQA_PROJ_KERNEL", kernel)
     gen = torch.Generator().manual_seed(B + K + N)
     x = torch.randn(B, K, generator=gen).to(torch.bfloat16)
     W = (torch.randn(K, N, generator=gen) * K ** -0.5).to(torch.bfloat16)
     ws = None
-    if split:
+    if kernel != "column":
         ws = torch.empty(gqa.project_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
     out = gqa.out_project(x.cuda(), W.cuda(), workspace=ws)
     gqa.get_status()

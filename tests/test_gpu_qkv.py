@@ -4,6 +4,10 @@ q and the appended k/v rows are compared with the fp64 oracle (bf16 inputs,
 fp32 accumulation, one rounding: the bf16 tolerance); every other cache
 position must be bit-identical to its input, and seqlens_out = seqlens + 1
 except for full caches, which get no append and flag GQA_ERR_SEQLEN.
+
+Two kernels can run a projection: the column-block kernel and the split-K
+kernel (with a workspace).  GQA_PROJ_KERNEL, read on every call, forces one,
+so each test runs both.
 """
 import pytest
 import torch
@@ -18,6 +22,9 @@ pytestmark = pytest.mark.gpu
 def _workspace(gqa, x):
     n = gqa.project_workspace_bytes((x.H + 2 * x.G) * x.d_h, x.d)
     return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+KERNELS = ["column", "split"]
 
 
 def run_and_check(gqa, x, expect_full=False, split=False):
@@ -53,31 +60,35 @@ def run_and_check(gqa, x, expect_full=False, split=False):
     (33, 256, 8, 8, 64, 10, [i % 10 for i in range(33)]),   # two launches, G = H (MHA)
     (5, 128, 32, 1, 128, 4, [3, 0, 1, 2, 3]),                # MQA
 ])
-@pytest.mark.parametrize("split", [False, True], ids=["column_blocks", "split_k"])
-def test_qkv_append_small(gqa, B, d, H, G, d_h, T, seqlens, split):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_qkv_append_small(gqa, monkeypatch, B, d, H, G, d_h, T, seqlens, kernel):
+    monkeypatch.setenv("GQA_PROJ_KERNEL", kernel)
     x = gi.qkv_inputs(B, d, H, G, d_h, T, seed=B + d, seqlens=seqlens)
-    run_and_check(gqa, x, split=split)
+    run_and_check(gqa, x, split=kernel == "split")
 
 
-@pytest.mark.parametrize("split", [False, True], ids=["column_blocks", "split_k"])
-def test_qkv_append_full_cache_is_not_written(gqa, split):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_qkv_append_full_cache_is_not_written(gqa, monkeypatch, kernel):
+    monkeypatch.setenv("GQA_PROJ_KERNEL", kernel)
     x = gi.qkv_inputs(4, 256, 8, 2, 64, 6, seed=3, seqlens=[6, 2, 6, 5])
-    run_and_check(gqa, x, expect_full=True, split=split)
+    run_and_check(gqa, x, expect_full=True, split=kernel == "split")
 
 
-@pytest.mark.parametrize("split", [False, True], ids=["column_blocks", "split_k"])
-def test_qkv_append_llama2_7b_full(gqa, split):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_qkv_append_llama2_7b_full(gqa, monkeypatch, kernel):
     """B=16, d=4096, H=32, G=8, d_h=128, T_cap=4096 (last free slot)."""
+    monkeypatch.setenv("GQA_PROJ_KERNEL", kernel)
     x = gi.workload_inputs("qkv_append_llama2_7b")
-    run_and_check(gqa, x, split=split)
+    run_and_check(gqa, x, split=kernel == "split")
 
 
-def test_split_k_is_deterministic_and_graph_replayable(gqa):
+def test_split_k_is_deterministic_and_graph_replayable(gqa, monkeypatch):
     """The split-K kernel adds a block's partial sums in slot order whichever CTA
     finishes last, and resets the block counters for the next call: repeated
     calls, and one call captured in a CUDA graph and replayed with h changed in
     place, give the bits of eager calls."""
     # 48 column blocks: each is split over three CTAs on a 148-SM part
+    monkeypatch.setenv("GQA_PROJ_KERNEL", "split")
     x = gi.qkv_inputs(16, 4096, 16, 4, 128, 8, seed=21, seqlens=[3] * 16)
     h, wq, wk, wv = x.h.cuda(), x.W_Q.cuda(), x.W_K.cuda(), x.W_V.cuda()
     kc, vc, sl = x.k_cache.cuda(), x.v_cache.cuda(), x.seqlens.cuda()
@@ -98,9 +109,11 @@ def test_split_k_is_deterministic_and_graph_replayable(gqa):
         h.copy_(torch.randn(h.shape, generator=gen).to(torch.bfloat16))
         graph.replay()
         got = q.clone()
-        eager = gqa.qkv_append(h, wq, wk, wv, kc.clone(), vc.clone(), sl)[0]  # column-block kernel
         eager_split = gqa.qkv_append(h, wq, wk, wv, kc.clone(), vc.clone(), sl,
                                      workspace=_workspace(gqa, x))[0]
+        monkeypatch.setenv("GQA_PROJ_KERNEL", "column")
+        eager = gqa.qkv_append(h, wq, wk, wv, kc.clone(), vc.clone(), sl)[0]
+        monkeypatch.setenv("GQA_PROJ_KERNEL", "split")
         torch.cuda.synchronize()
         gqa.get_status()
         assert torch.equal(got, eager_split), "replay %d" % i
