@@ -44,15 +44,26 @@ ROW_WORKLOADS = ["tiny_decode_fp32", "llama2_70b_ragged_decode"] + \
                                                                 "layer_decode_llama2_7b"]
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
-# kernel, in bytes, each from one ncu capture of the kernel as it is now (the
-# summaries under profiles/ give the commands); a workload missing here has no
-# capture of its current kernel, and its traffic is reported as null.
+# kernel, in bytes, each from one single-pass ncu capture of that kernel as it
+# is now, on the full workload (the ncu summaries give the commands); for the
+# layer step, the sum over its four kernels (Q/K/V projection, decode split,
+# combine, W_O projection).  A workload missing here has no capture of its
+# current kernel, and its traffic is reported as null.
 NCU_TRAFFIC = {
-    "llama2_7b_decode": 272493056,      # warp-MMA split kernel, full workload
-    "long_ctx_decode_G1": 273029376,    # tcgen05 split kernel, full workload
-    "causal_prefill": 397575168,        # B=1, S=4096 case, scaled by 4 (traffic grows with the q/k/v/out bytes)
-    "meanpool_init": 289036800,         # full workload
-    "qkv_append_llama2_7b": 50488832,   # full workload
+    "llama2_7b_decode": 271766784,                     # warp-MMA split kernel
+    "llama2_70b_ragged_decode": 658599680,
+    "llama2_70b_ragged_decode_window4096": 462243840,
+    "long_ctx_decode_G1": 271518464,                   # tcgen05 split kernel
+    "long_ctx_decode_G2": 539975680,
+    "long_ctx_decode_G4": 1076642816,                  # warp-MMA split kernel from here on
+    "long_ctx_decode_G8": 2150617600,
+    "long_ctx_decode_G16": 4298365440,
+    "long_ctx_decode_G32": 8593204992,
+    "causal_prefill": 734912768,
+    "causal_prefill_window4096": 559403520,
+    "meanpool_init": 288286208,
+    "qkv_append_llama2_7b": 50485248,
+    "layer_decode_llama2_7b": 357017088,
 }
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
