@@ -146,21 +146,6 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
 #endif
 constexpr int kExpPolyOf8 = GQA_PREFILL_EXP_POLY_OF_8;
 
-// 1: a tile's exponentials start from the running max before the tile's own
-// max is known (see the softmax); 0: max first, then the exponentials.
-#ifndef GQA_PREFILL_SPEC_MAX
-#define GQA_PREFILL_SPEC_MAX 0
-#endif
-constexpr bool kSpecMax = GQA_PREFILL_SPEC_MAX != 0;
-
-// 1: as GQA_PREFILL_SPEC_MAX, and the tile's scores are loaded from tensor
-// memory 32 at a time, each chunk's load overlapping the previous chunk's
-// exponentials.
-#ifndef GQA_PREFILL_PIPE
-#define GQA_PREFILL_PIPE 0
-#endif
-constexpr bool kPipe = GQA_PREFILL_PIPE != 0;
-
 // Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64_t limit) {
     const bool ok = mbar_wait(bar, parity, limit);
@@ -407,32 +392,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             };
-            // Pipelined tile (kPipe, every tile after a row's first, P in one bf16
-            // term): the exponentials start from the running max m as soon as the
-            // first 32 scores are in registers, while the next 32 load, and the
-            // tile's max is kept on the fly for the rescale check after the pass.
-            const bool pipe = kPipe && jj > 0 && !split_p;
-            if (!pipe) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, sr[c]);
-                tc::wait_ld();
+            for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, sr[c]);
+            tc::wait_ld();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tc::hold32(sr[c]);
-                    mask_chunk(c);
-                }
+            for (int c = 0; c < 4; ++c) {
+                tc::hold32(sr[c]);
+                mask_chunk(c);
             }
             // Row maximum of the raw scores (the scale is positive), with eight
             // independent partial maxima instead of one 128-long chain.
             float mx8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-            if (!pipe) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[c][e]));
-            }
+                for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[c][e]));
             // P = 2^(s * scale_log2 - m) in bf16 pairs over the first 64 columns of
             // this S block; the exponent argument is formed two at a time (packed
             // fp32 FMA) and the row sum kept in four packed partial sums.
@@ -498,94 +474,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return sum;
             };
-            // the pipelined pass: P from the running max, chunk by chunk
-            float rs_pipe = 0.f;
-            if (pipe) {
-                const float mu = m == -INFINITY ? 0.f : m;
-                const uint64_t nm2 = f32x2_pack(-mu, -mu);
-                uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
-                tc::ld32(tS, sr[0]);
-                tc::wait_ld();
-                tc::hold32(sr[0]);
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    if (c4 < 3) tc::ld32(tS + (c4 + 1) * 32, sr[c4 + 1]);  // lands while this chunk runs
-                    mask_chunk(c4);
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float a = __uint_as_float(sr[c4][2 * e]), b = __uint_as_float(sr[c4][2 * e + 1]);
-                        mx8[(2 * e) & 7] = fmaxf(mx8[(2 * e) & 7], a);
-                        mx8[(2 * e + 1) & 7] = fmaxf(mx8[(2 * e + 1) & 7], b);
-                        const uint64_t x2 = f32x2_fma(f32x2_pack(a, b), sc2, nm2);
-                        float p0, p1;
-                        if ((e & 7) < kExpPolyOf8) {
-                            f32x2_unpack(exp2_poly_x2(x2), p0, p1);
-                        } else {
-                            float x0, x1;
-                            f32x2_unpack(x2, x0, x1);
-                            p0 = fast_exp2(x0);
-                            p1 = fast_exp2(x1);
-                        }
-                        rs2[e & 3] = f32x2_add(rs2[e & 3], f32x2_pack(p0, p1));
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tc::st16(tS + c4 * 16, pk);  // over S columns already in registers
-                    if (c4 < 3) {
-                        tc::wait_ld();
-                        tc::hold32(sr[c4 + 1]);
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float a0, a1;
-                    f32x2_unpack(rs2[i], a0, a1);
-                    rs_pipe += a0 + a1;
-                }
-            }
             const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
             float alpha = 1.f;
             bool rescale = false;
-            // With kSpecMax the running max m, which only moves when a tile's max
-            // exceeds it by more than 8, is used before this tile's max is known,
-            // so the exponentials need not wait for the max; a warp with a row
-            // whose max did move redoes the pass (its other rows recompute the same
-            // values).  Otherwise the max is settled first.
-            const bool spec = (kSpecMax || pipe) && jj > 0 && !split_p;
-            if (!spec) {
-                if (jj == 0) {
-                    m = mx;  // -inf when a sliding window hides this tile from the row
-                } else {
-                    const float mn = fmaxf(m, mx);
-                    const bool need = mn > m + 8.f;
-                    rescale = __any_sync(0xffffffffu, need);
-                    if (need) {
-                        alpha = fast_exp2(m - mn);
-                        m = mn;
-                        l *= alpha;
-                    }
-                }
-            }
-            float rs;
-#pragma unroll 1
-            for (int pass = 0;; ++pass) {
-                if (pipe && pass == 0)
-                    rs = rs_pipe;  // the pipelined pass above
-                else
-                    rs = exp_pass(m);
-                if (!spec || pass > 0) break;
+            if (jj == 0) {
+                m = mx;  // -inf when a sliding window hides this tile from the row
+            } else {
                 const float mn = fmaxf(m, mx);
-                const bool need = mn > m + 8.f;  // also when m was -inf and mn is not
+                const bool need = mn > m + 8.f;
                 rescale = __any_sync(0xffffffffu, need);
-                if (!rescale) break;
                 if (need) {
                     alpha = fast_exp2(m - mn);
                     m = mn;
                     l *= alpha;
                 }
-                tc::wait_st();
             }
+            const float rs = exp_pass(m);
             if (rescale) {  // O was last written by the P.V of tile j-1, complete by now
 #pragma unroll 1
                 for (int c = 0; c < D / 16; ++c) {
