@@ -540,8 +540,15 @@ __global__ void __launch_bounds__(kThreadsF32)
 // (see run_combine).
 constexpr int kCombBatch = 8;
 
+// One block per SM is all the launch bounds ask for, so the compiler keeps
+// the merge loop in registers (94 at d_h = 128, no spills).  Left to its own
+// choice it fitted the 16-warp combine into 64 registers with 136 bytes of
+// spills, and that combine then also fitted next to the tcgen05 split kernel
+// on every SM, where its polling slowed the split: graph-timed, the G = 2
+// long-context step took 99-104 us that way against 89-90 us with these
+// bounds (7B-shaped step: 47.6 us either way).
 template <int D, bool BF16_OUT, int NW>
-__global__ void __launch_bounds__(NW * 32) decode_combine(const DecodeParams p, int C) {
+__global__ void __launch_bounds__(NW * 32, 1) decode_combine(const DecodeParams p, int C) {
     constexpr int PER = D / 32;
     __shared__ float red_m[NW], red_l[NW];
     __shared__ int red_bad[NW];
