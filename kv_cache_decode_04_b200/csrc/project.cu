@@ -222,14 +222,14 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 }
 
 // ------------------------------------------------------------------------
-// Split-K variant for every SM.  The column-block kernel above gives each
-// 64-column block of the weights one CTA, which leaves SMs idle whenever
-// there are fewer blocks than SMs (96 for the Llama-2-7B Q/K/V projection, 64
-// for its W_O).  Here each block's 128-row K tiles are also cut into ks equal
-// row ranges: items (block cb, range s), item = s * nblocks + cb, taken by
-// CTA item mod gridDim.x in increasing order.  The host takes
-// ks = floor(SMs / blocks), so every item has a CTA of its own in one wave
-// (split_plan below).  Items of the same
+// Split-K variant for projections with few column blocks.  The column-block
+// kernel above gives each 64-column block of the weights one CTA, which
+// leaves most SMs idle when there are only a few blocks.  Here each block's
+// 128-row K tiles are also cut into ks equal row ranges: items (block cb,
+// range s), item = s * nblocks + cb, taken by CTA item mod gridDim.x in
+// increasing order.  The host takes ks = floor(SMs / blocks), so every item
+// has a CTA of its own in one wave, and uses this kernel only when ks >= 4
+// (split_plan and proj_kernel below).  Items of the same
 // range start together on different CTAs, so the CTAs running at one time
 // read the same weight rows (different column blocks): the DRAM pages a row
 // spans are read by many CTAs at once, as in the column-block kernel.  (Equal
