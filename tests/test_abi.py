@@ -71,3 +71,36 @@ def test_prefill_and_meanpool_reject_bad_arguments_on_host():
     # outputs overlapping the inputs
     assert L.gqa_meanpool_kv(1 << 20, 1 << 24, (1 << 20) + 64, 1 << 28, 8, 2, 4, 4,
                              gqa.GQA_BF16, None) == -1
+
+
+def _qkv_rc(**kw):
+    a = dict(h=1 << 20, wq=1 << 21, wk=1 << 22, wv=1 << 23, q=1 << 24, kc=1 << 25, vc=1 << 26,
+             sl=1 << 27, slo=1 << 28, B=4, d=256, H=8, G=2, d_h=128, T=16, dt=gqa.GQA_BF16)
+    a.update(kw)
+    return gqa.lib.gqa_qkv_append(a["h"], a["wq"], a["wk"], a["wv"], a["q"], a["kc"], a["vc"], a["sl"], a["slo"],
+                                  a["B"], a["d"], a["H"], a["G"], a["d_h"], a["T"], a["dt"], None, 0, None)
+
+
+def test_projections_reject_bad_arguments_on_host():
+    assert _qkv_rc(G=3) == -1                       # G does not divide H
+    assert _qkv_rc(B=0) == -1
+    assert _qkv_rc(d=0) == -1
+    assert _qkv_rc(T=0) == -1
+    assert _qkv_rc(h=None) == -1
+    assert _qkv_rc(slo=(1 << 27) + 4) == -1        # seqlens_out overlaps seqlens
+    assert _qkv_rc(dt=gqa.GQA_F32) == -2
+    assert _qkv_rc(d_h=96) == -2
+    assert _qkv_rc(d=200) == -2                     # d not a multiple of 128
+    assert _qkv_rc(wq=(1 << 21) + 8) == -3          # weights must be 16-byte aligned
+    assert _qkv_rc(G=3) == -1 and "divide" in gqa.lib.gqa_last_error_string().decode()
+    L = gqa.lib
+    x, w, o = 1 << 20, 1 << 24, 1 << 28
+    assert L.gqa_out_project(x, w, o, 0, 256, 128, gqa.GQA_BF16, None, 0, None) == -1
+    assert L.gqa_out_project(None, w, o, 4, 256, 128, gqa.GQA_BF16, None, 0, None) == -1
+    assert L.gqa_out_project(x, w, o, 4, 256, 128, gqa.GQA_F32, None, 0, None) == -2
+    assert L.gqa_out_project(x, w, o, 4, 200, 128, gqa.GQA_BF16, None, 0, None) == -2   # K % 128
+    assert L.gqa_out_project(x, w, o, 4, 256, 96, gqa.GQA_BF16, None, 0, None) == -2    # N % 64
+    assert L.gqa_out_project(x + 4, w, o, 4, 256, 128, gqa.GQA_BF16, None, 0, None) == -3
+    # the layer step needs the post-append lengths
+    assert L.gqa_layer_decode_step(x, w, w, w, w, o, o, x, None, 0.1, 0, o, 4, 256, 8, 2, 128, 16,
+                                   gqa.GQA_BF16, None, 0, None) == -1
