@@ -54,6 +54,7 @@ def test_decode_rejects_bad_arguments_on_host():
     assert _decode_rc(d_h=96)[0] == -2                     # not built
     assert _decode_rc(dt=7)[0] == -2
     assert _decode_rc(H=130, G=2)[0] == -2                 # bf16 group of 65 heads
+    assert _decode_rc(B=8193)[0] == -2                     # above the largest batch built for
     assert _decode_rc(k=24)[0] == -3                       # misaligned
     rc, msg = _decode_rc(G=3)
     assert "divide" in msg

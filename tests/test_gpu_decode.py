@@ -244,3 +244,18 @@ def test_workspace_initial_contents_do_not_matter(gqa, fill):
         out = gqa.decode(q, k, v, sl, x.scale, workspace=ws)
         gqa.get_status()
         assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_largest_batch(gqa, dtype):
+    """B = 8192, the largest batch the calls take: the tile prefix over 8192
+    lengths (chunked over the block's threads), shares that cross hundreds of
+    sequences, and empty caches among them."""
+    gen = torch.Generator().manual_seed(8192)
+    seqlens = torch.randint(0, 17, (8192,), generator=gen).tolist()
+    x = gi.decode_inputs(8192, 8, 2, 64, 16, dtype, seed=8192, seqlens=seqlens)
+    got = run_decode(gqa, x)
+    ref = oracle.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    assert_close(got, ref, dtype)
+    empty = [b for b, t in enumerate(seqlens) if t == 0]
+    assert empty and torch.equal(got[empty], torch.zeros_like(got[empty]))
