@@ -9,11 +9,11 @@
 // ~210 TFLOP/s of dense contraction, more than warp-level MMAs sustain next to
 // the softmax, so here both products run on tcgen05.
 //
-// Tensor-core cost: a tcgen05.mma with M = 128, K = 16 and N <= 128 occupies
-// the tensor pipe for about 96 cycles on B200 whatever N is (measured), so the
-// instruction count, not the flops, is what this kernel has to keep small.
+// Tensor-core cost: a tcgen05.mma with M = 128 and K = 16 takes 56 SM cycles
+// at N = 64 and 64 at N = 128 when one thread streams them (measured on B200),
+// so below N = 128 the instruction count matters as much as the flops.
 // Tiles are 128 positions: S = Q K^T is 8 instructions of N = 128 and P.V 8
-// of N = d_h per tile, about half the HBM time of the tile's 64 KB.
+// of N = d_h per tile, about a third of the HBM time of the tile's 64 KB.
 //
 // Rows of the M = 128 tile: the group's H/G query rows, replicated NREP times
 // (4 copies of 32 rows for H/G <= 32, 2 copies of 64 rows above).  Copy k is
