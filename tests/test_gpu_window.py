@@ -42,6 +42,20 @@ def test_prefill_window(gqa, S, W):
     assert_close(out.cpu(), ref, torch.bfloat16)
 
 
+@pytest.mark.parametrize("S,W,H,G,d_h", [
+    (1024, 257, 8, 2, 128),  # one key past the two-term-P threshold (W <= 256)
+    (500, 130, 6, 2, 64),    # r = 3 (a lone head per group) at d_h = 64
+    (300, 64, 4, 4, 64),     # G = H (MHA) with a window inside one tile
+    (777, 200, 10, 2, 128),  # r = 5, ragged S
+])
+def test_prefill_window_group_sizes_and_head_dims(gqa, S, W, H, G, d_h):
+    x = gi.prefill_inputs(1, S, H, G, d_h, torch.bfloat16, seed=S + W + d_h)
+    out = gqa.prefill_causal(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.scale, window=W)
+    gqa.get_status()
+    ref = oracle.gqa_prefill_causal(x.q, x.k, x.v, x.scale, window=W)
+    assert_close(out.cpu(), ref, torch.bfloat16)
+
+
 def test_prefill_window_4096_full_workload(gqa):
     """B=2, S=8192, H=64, G=8 with a 4096-key window: every tile edge of one
     (b, head) and 1,024 random rows; strict form on rows below 0.5."""
