@@ -31,9 +31,12 @@
  *     status bit (GQA_ERR_INDEX from gqa_get_status).  Same ABI and results.
  *   - Results are deterministic: the same inputs and launch give the same bits.
  *   - Kernels are launched as programmatic dependents: a call's set-up may
- *     overlap the end of the work before it on `stream`, but no kernel reads
- *     an input before that work has completed, so ordinary stream ordering
- *     holds.  Calls can be captured in CUDA graphs.
+ *     overlap the end of the work before it on `stream`, but no kernel uses an
+ *     input's value before that work has completed, so ordinary stream
+ *     ordering holds.  (The decode kernels read seqlens early to guess their
+ *     first cache tiles and ask L2 to fetch them: a hint, which a value still
+ *     being written can make wasted but cannot make wrong.)  Calls can be
+ *     captured in CUDA graphs.
  */
 #ifndef GQA_H
 #define GQA_H

@@ -134,6 +134,12 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, u
 
 // ------------------------------------------------------------ TMA
 
+// Asks L2 to fetch [src, src + bytes) (both 16-byte multiples); a hint, no
+// data reaches the SM and nothing waits for it.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }

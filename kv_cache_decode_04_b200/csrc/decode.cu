@@ -116,9 +116,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kCWarps && lane == 0) {
-        tma_prefetch_desc(&tmk);
-        tma_prefetch_desc(&tmv);
+    if (warp == kCWarps) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+        }
+        // 8 tiles (4 ring fills): graph-replayed A/Bs put 8 ahead of 2, 4, 12 and
+        // 16 on the 7B- and 70B-shaped steps, and level with none on long rows
+        dec::warm_first_tiles<kTile>(p, lane, 8, D * 2);
     }
     pdl_wait_primary();  // inputs written by the kernels before this one are visible
     const unsigned long long gen = dec::call_generation(p);
@@ -873,6 +878,7 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap *tmk, const CUt
     p.T_cap = a.T_cap;
     p.timeout_ns = a.timeout_ns;
     p.window = a.window;
+    p.warm = a.warm;
     p.ws_flag = reinterpret_cast<unsigned long long *>(ws + L.off_flag);
     p.ws_hdr = reinterpret_cast<unsigned long long *>(ws + L.off_hdr);
     p.n_rec = L.n_rec;

@@ -29,12 +29,15 @@ struct DecodeParams {
     float2 *ws_ml;  // [n_rec * r]: (max in log2 units, sum)
     float *ws_o;    // [n_rec * r * d_h]: unnormalised outputs
     long long n_rec;  // records the workspace holds (the debug build's index checks)
-    const float *k32, *v32;  // fp32 path only
+    // Cache bases, typed for the fp32 path; the bf16 kernels use them only for
+    // L2 prefetch hints (their loads go through tensor maps).
+    const float *k32, *v32;
     unsigned *status;
     float scale_log2;
     int B, H, G, r, T_cap;
     unsigned long long timeout_ns;
     int window;  // > 0: attend over the last `window` cached positions only
+    int warm;    // nonzero: warm L2 with the first tiles before griddepcontrol.wait
     // Completion flags, [1 + records]: flag 0 = the tile prefix ws_cu, flag 1 + i
     // = record i.  A flag holds the generation of the call that completed it.
     unsigned long long *ws_flag;
@@ -170,6 +173,45 @@ __device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, b
 
 // Position in the tile line: sequence b, KV head g, tile j of the segment,
 // tiles per segment of b.
+// L2 warm-up for a split kernel's first tiles, issued by one warp before
+// griddepcontrol.wait, so that the cache reads start while the kernel before
+// this one ends.  seqlens may be an output of that kernel and is read here
+// only to guess this CTA's share (B <= 32: one warp scans it); a stale guess
+// costs bandwidth, never correctness, since the loads proper come after the
+// wait.  Prefetches up to `ntiles` tiles of TILE positions (row_bytes each)
+// from the start of the share, within its first segment.
+template <int TILE>
+__device__ __forceinline__ void warm_first_tiles(const DecodeParams &p, int lane, int ntiles, int row_bytes) {
+    if (!p.warm || p.B > 32) return;
+    int T = 0, n = 0;
+    if (lane < p.B) {
+        T = clamp_len(*reinterpret_cast<const volatile int32_t *>(p.seqlens + lane), p.T_cap);
+        n = p.G * ((attended_len(T, p) + TILE - 1) / TILE);
+    }
+    int incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    const int u0 = (int)((long long)blockIdx.x * total / gridDim.x);
+    const int u1 = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
+    const int excl = incl - n;
+    if (lane >= p.B || u0 >= u1 || u0 < excl || u0 >= incl) return;  // not the lane holding u0
+    const int len = attended_len(T, p), start = T - len, nt = (len + TILE - 1) / TILE;
+    const uint8_t *kb = reinterpret_cast<const uint8_t *>(p.k32);
+    const uint8_t *vb = reinterpret_cast<const uint8_t *>(p.v32);
+    int idx = u0 - excl;  // tile of this sequence's G segments, g-major
+    for (int k = 0; k < ntiles && u0 + k < u1 && idx < p.G * nt; ++k, ++idx) {
+        const int g = idx / nt, j = idx - g * nt;
+        const int ntok = min(TILE, len - j * TILE);
+        const size_t row = ((size_t)lane * p.G + g) * p.T_cap + start + (size_t)j * TILE;
+        prefetch_l2(kb + row * row_bytes, (uint32_t)(ntok * row_bytes));
+        prefetch_l2(vb + row * row_bytes, (uint32_t)(ntok * row_bytes));
+    }
+}
+
 struct Cursor {
     int b, g, j, ntb;
 };

@@ -187,9 +187,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 4 && lane == 0) {
-        tma_prefetch_desc(&tmk);
-        tma_prefetch_desc(&tmv);
+    if (warp == 4) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+        }
+        // one ring's worth: deeper warm-ups measured no better here
+        warm_first_tiles<kTT>(p, lane, STAGES, D * 2);
     }
     if (warp == 5) {
         tc::tmem_alloc(tmem_slot, kTcTmemCols);

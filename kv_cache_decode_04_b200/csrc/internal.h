@@ -27,6 +27,7 @@ struct DecodeArgs {
     int num_sms;
     int force_ctas;  // >0: use this many split CTAs (tests of the split logic)
     int window;      // >0: sliding window of the last `window` cached positions
+    int warm;        // nonzero: the split kernels warm L2 with their first tiles early
 };
 
 // Workspace layout, all offsets 256-byte aligned.  The first 256 bytes are a
