@@ -171,15 +171,13 @@ __device__ int build_tile_prefix(const DecodeParams &p, int *cu, int *scratch, b
     return cu[p.B];
 }
 
-// Position in the tile line: sequence b, KV head g, tile j of the segment,
-// tiles per segment of b.
 // L2 warm-up for a split kernel's first tiles, issued by one warp before
 // griddepcontrol.wait, so that the cache reads start while the kernel before
 // this one ends.  seqlens may be an output of that kernel and is read here
 // only to guess this CTA's share (B <= 32: one warp scans it); a stale guess
 // costs bandwidth, never correctness, since the loads proper come after the
 // wait.  Prefetches up to `ntiles` tiles of TILE positions (row_bytes each)
-// from the start of the share, within its first segment.
+// from the start of the share, within the sequence the share starts in.
 template <int TILE>
 __device__ __forceinline__ void warm_first_tiles(const DecodeParams &p, int lane, int ntiles, int row_bytes) {
     if (!p.warm || p.B > 32) return;
@@ -212,6 +210,8 @@ __device__ __forceinline__ void warm_first_tiles(const DecodeParams &p, int lane
     }
 }
 
+// Position in the tile line: sequence b, KV head g, tile j of the segment,
+// tiles per segment of b.
 struct Cursor {
     int b, g, j, ntb;
 };
