@@ -61,7 +61,7 @@ NCU_TRAFFIC = {
     "long_ctx_decode_G32": 8594387456,
     "causal_prefill": 734912768,
     "causal_prefill_window4096": 559403520,
-    "meanpool_init": 288286208,
+    "meanpool_init": 274089216,
     "qkv_append_llama2_7b": 50485248,
     "layer_decode_llama2_7b": 356922368,
 }

@@ -76,6 +76,22 @@ __global__ void __launch_bounds__(256) meanpool_vec(const uint4 *__restrict__ wk
     const bool pow2 = (r & (r - 1)) == 0;
     auto mean = [&](double a) { return pow2 ? __dmul_rn(a, inv_r) : __ddiv_rn(a, dr); };
     const int H = (int)(r * (out_vec / n_vec));
+    {   // L2 hint for this thread's first vectors, before the wait for the work ahead
+        // (addresses only: the values are read after the wait)
+        const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+        if (idx < total) {
+            const bool is_v = idx >= out_vec;
+            const long long v = is_v ? idx - out_vec : idx;
+            const long long g = v / n_vec, e = v - g * n_vec;
+            if (g * r + r <= H) {
+                const uint4 *src = (is_v ? wv : wk) + (g * r) * n_vec + e;
+                for (int j = 0; j < r; ++j)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(src + (long long)j * n_vec));
+            }
+        }
+    }
+    pdl_wait_primary();       // inputs written by the work before this kernel are visible
+    pdl_launch_dependents();  // the next kernel may set up while this one streams
     for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
         const bool is_v = idx >= out_vec;
@@ -125,6 +141,8 @@ __global__ void __launch_bounds__(256) meanpool_scalar(const void *wk, const voi
                                                        void *ov, int r, long long n,
                                                        long long out_n, const float *wts, int sel,
                                                        unsigned *status) {
+    pdl_wait_primary();
+    pdl_launch_dependents();
     const long long total = 2 * out_n;
     const double dr = (double)r, inv_r = 1.0 / dr;
     const bool pow2 = (r & (r - 1)) == 0;
@@ -166,6 +184,24 @@ __global__ void __launch_bounds__(256) meanpool_scalar(const void *wk, const voi
     }
 }
 
+// Launched as programmatic dependents: the kernels ask L2 for their first
+// inputs (a hint) and then wait for the work ahead of them on the stream
+// before they read or write anything.
+cudaLaunchConfig_t pdl_config(unsigned blocks, int threads, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    return cfg;
+}
+void pdl_attr(cudaLaunchConfig_t &cfg, cudaLaunchAttribute (&attr)[1]) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+}
+
 template <int MODE>
 cudaError_t launch_mode(const void *wk, const void *wv, void *ok, void *ov, int H, int G, long long n, bool bf16,
                         bool aligned, int num_sms, const float *wts, int sel, unsigned *status,
@@ -180,14 +216,22 @@ cudaError_t launch_mode(const void *wk, const void *wv, void *ok, void *ov, int 
         long long blocks = (2 * out_vec + threads - 1) / threads;
         if (blocks > cap) blocks = cap;
         auto kern = bf16 ? meanpool_vec<true, MODE> : meanpool_vec<false, MODE>;
-        kern<<<(unsigned)blocks, threads, 0, st>>>(static_cast<const uint4 *>(wk), static_cast<const uint4 *>(wv),
-                                                   static_cast<uint4 *>(ok), static_cast<uint4 *>(ov), r, n_vec,
-                                                   out_vec, wts, sel, status);
+        cudaLaunchConfig_t cfg = pdl_config((unsigned)blocks, threads, st);
+        cudaLaunchAttribute attr[1];
+        pdl_attr(cfg, attr);
+        cudaError_t le = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint4 *>(wk), static_cast<const uint4 *>(wv),
+                                            static_cast<uint4 *>(ok), static_cast<uint4 *>(ov), r, n_vec, out_vec, wts,
+                                            sel, status);
+        if (le != cudaSuccess) return le;
     } else {
         long long blocks = (2 * out_elems + threads - 1) / threads;
         if (blocks > cap) blocks = cap;
         auto kern = bf16 ? meanpool_scalar<true, MODE> : meanpool_scalar<false, MODE>;
-        kern<<<(unsigned)blocks, threads, 0, st>>>(wk, wv, ok, ov, r, n, out_elems, wts, sel, status);
+        cudaLaunchConfig_t cfg = pdl_config((unsigned)blocks, threads, st);
+        cudaLaunchAttribute attr[1];
+        pdl_attr(cfg, attr);
+        cudaError_t le = cudaLaunchKernelEx(&cfg, kern, wk, wv, ok, ov, r, n, out_elems, wts, sel, status);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
