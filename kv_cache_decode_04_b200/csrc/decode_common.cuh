@@ -183,7 +183,9 @@ __device__ __forceinline__ void warm_first_tiles(const DecodeParams &p, int lane
     if (!p.warm || p.B > 32) return;
     int T = 0, n = 0;
     if (lane < p.B) {
-        T = clamp_len(*reinterpret_cast<const volatile int32_t *>(p.seqlens + lane), p.T_cap);
+        // cached at L2 only (ld.global.cg): no L1 line of a value that may be
+        // about to change outlives the wait
+        T = clamp_len(__ldcg(p.seqlens + lane), p.T_cap);
         n = p.G * ((attended_len(T, p) + TILE - 1) / TILE);
     }
     int incl = n;

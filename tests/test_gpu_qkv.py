@@ -131,3 +131,26 @@ def test_qkv_then_decode_sees_the_new_token(gqa):
     ref = oracle.gqa_decode(q.cpu(), kc.cpu(), vc.cpu(), sl_out.cpu(), 128 ** -0.5)
     assert_close(out.cpu(), ref, torch.bfloat16)
     assert sl_out.cpu().tolist() == [11, 40]
+
+
+def test_append_then_decode_chain_across_tile_boundaries(gqa):
+    """Twenty append -> decode rounds back to back on one stream, each decode over the
+    lengths the append before it has just written (seqlens_out), starting one
+    position short of a 64-token tile boundary: every round must see its new token."""
+    x = gi.qkv_inputs(2, 256, 8, 2, 128, 160, seed=21, seqlens=[63, 127])
+    kc, vc = x.k_cache.cuda(), x.v_cache.cuda()
+    h, wq, wk, wv = x.h.cuda(), x.W_Q.cuda(), x.W_K.cuda(), x.W_V.cuda()
+    sl = x.seqlens.cuda()
+    outs, qs, lens = [], [], []
+    for _ in range(20):
+        q, sl_out = gqa.qkv_append(h, wq, wk, wv, kc, vc, sl)
+        outs.append(gqa.decode(q, kc, vc, sl_out, 128 ** -0.5))
+        qs.append(q)
+        lens.append(sl_out)
+        sl = sl_out
+    gqa.get_status()
+    kc_c, vc_c = kc.cpu(), vc.cpu()
+    for i, (out, q, L) in enumerate(zip(outs, qs, lens)):
+        assert L.cpu().tolist() == [64 + i, 128 + i]
+        ref = oracle.gqa_decode(q.cpu(), kc_c, vc_c, L.cpu(), 128 ** -0.5)
+        assert_close(out.cpu(), ref, torch.bfloat16)
