@@ -50,20 +50,20 @@ ROW_WORKLOADS = ["tiny_decode_fp32", "llama2_70b_ragged_decode"] + \
 # combine, W_O projection).  A workload missing here has no capture of its
 # current kernel, and its traffic is reported as null.
 NCU_TRAFFIC = {
-    "llama2_7b_decode": 272031488,                     # warp-MMA split kernel
-    "llama2_70b_ragged_decode": 659014656,
-    "llama2_70b_ragged_decode_window4096": 462499840,
-    "long_ctx_decode_G1": 271576576,                   # tcgen05 split kernel
-    "long_ctx_decode_G2": 540104192,
-    "long_ctx_decode_G4": 1077687808,                  # warp-MMA split kernel from here on
-    "long_ctx_decode_G8": 2151217920,
-    "long_ctx_decode_G16": 4299063040,
-    "long_ctx_decode_G32": 8594387456,
+    "llama2_7b_decode": 271878400,                     # warp-MMA split kernel
+    "llama2_70b_ragged_decode": 658844672,
+    "llama2_70b_ragged_decode_window4096": 462055936,
+    "long_ctx_decode_G1": 271545088,                   # tcgen05 split kernel
+    "long_ctx_decode_G2": 539985664,
+    "long_ctx_decode_G4": 1079909120,                  # warp-MMA split kernel from here on
+    "long_ctx_decode_G8": 2151690240,
+    "long_ctx_decode_G16": 4299057152,
+    "long_ctx_decode_G32": 8595744256,
     "causal_prefill": 734912768,
     "causal_prefill_window4096": 559403520,
     "meanpool_init": 274089216,
     "qkv_append_llama2_7b": 50485248,
-    "layer_decode_llama2_7b": 356922368,
+    "layer_decode_llama2_7b": 358748928,
 }
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
