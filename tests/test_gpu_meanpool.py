@@ -136,3 +136,27 @@ def test_init_rejects_bad_selection(gqa):
         gqa.init_kv_heads(wk.cuda(), wv.cuda(), 2, mode="select", select=4)
     with pytest.raises(gqa.GQAError):
         gqa.init_kv_heads(wk.cuda(), wv.cuda(), 2, mode="weighted")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_meanpool_reads_what_the_kernel_before_wrote(gqa, dtype):
+    """The mean-pool kernels start as programmatic dependents and touch only
+    addresses before they wait: weights written by the kernel launched just
+    before them (here a torch elementwise kernel, alternating between two
+    contents) must be the ones they average."""
+    H, G, d_h, d = 16, 4, 64, 256
+    wk, wv = gi.meanpool_inputs(H, d_h, d, dtype=dtype, seed=5, std=0.5)
+    wk2, wv2 = gi.meanpool_inputs(H, d_h, d, dtype=dtype, seed=6, std=0.5)
+    dk, dv = torch.empty_like(wk).cuda(), torch.empty_like(wv).cuda()
+    srcs = [(wk.cuda(), wv.cuda()), (wk2.cuda(), wv2.cuda())]
+    outs = []
+    for i in range(6):
+        sk, sv = srcs[i % 2]
+        torch.mul(sv, 1, out=dv)   # an elementwise kernel writes the inputs ...
+        torch.mul(sk, 1, out=dk)
+        outs.append(gqa.meanpool_kv(dk, dv, G))  # ... and the mean-pool follows at once
+    gqa.get_status()
+    for i, (ok, ov) in enumerate(outs):
+        k, v = (wk, wv) if i % 2 == 0 else (wk2, wv2)
+        assert torch.equal(bits(ok.cpu()), bits(oracle.meanpool(k, G))), i
+        assert torch.equal(bits(ov.cpu()), bits(oracle.meanpool(v, G))), i
