@@ -62,8 +62,8 @@ NCU_TRAFFIC = {
     "causal_prefill": 734912768,
     "causal_prefill_window4096": 559403520,
     "meanpool_init": 274089216,
-    "qkv_append_llama2_7b": 50485248,
-    "layer_decode_llama2_7b": 358748928,
+    "qkv_append_llama2_7b": 50491136,
+    "layer_decode_llama2_7b": 357121280,
 }
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}

@@ -386,10 +386,16 @@ static int check_proj_workspace(void *workspace, size_t bytes, int ncols, int d,
     return GQA_OK;
 }
 
-int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V, void *q_out,
-                   void *k_cache, void *v_cache, const int32_t *seqlens, int32_t *seqlens_out, int B, int d,
-                   int H, int G, int d_h, int T_cap, gqa_dtype dt, void *workspace, size_t workspace_bytes,
-                   gqa_stream_t stream) {
+// warm: the column kernel asks L2 for its first weight tiles before the wait
+// for the work ahead of it (a hint).  The layer step turns it on: its Q/K/V
+// projection follows the previous step's W_O projection, which leaves most
+// SMs idle, and the 7B-shaped step went from 70.5 to 69.6 us.  Back to back
+// with itself, as in repeated standalone calls, it was slower (12.0 against
+// 11.7 us), so gqa_qkv_append leaves it off.
+static int qkv_append_impl(const void *h, const void *W_Q, const void *W_K, const void *W_V, void *q_out,
+                           void *k_cache, void *v_cache, const int32_t *seqlens, int32_t *seqlens_out, int B,
+                           int d, int H, int G, int d_h, int T_cap, gqa_dtype dt, void *workspace,
+                           size_t workspace_bytes, gqa_stream_t stream, bool warm) {
     t_err[0] = 0;
     int rc = check_dims(B, H, G, d_h);
     if (rc) return rc;
@@ -454,9 +460,18 @@ int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *
     a.workspace = workspace;
     a.num_sms = dev->num_sms;
     a.tag = next_tag();
+    a.warm = warm ? 1 : 0;
     cudaError_t e = gqa::launch_qkv_append(a, &tq, &tk, &tv, &th, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "qkv_append launch");
     return GQA_OK;
+}
+
+int gqa_qkv_append(const void *h, const void *W_Q, const void *W_K, const void *W_V, void *q_out,
+                   void *k_cache, void *v_cache, const int32_t *seqlens, int32_t *seqlens_out, int B, int d,
+                   int H, int G, int d_h, int T_cap, gqa_dtype dt, void *workspace, size_t workspace_bytes,
+                   gqa_stream_t stream) {
+    return qkv_append_impl(h, W_Q, W_K, W_V, q_out, k_cache, v_cache, seqlens, seqlens_out, B, d, H, G, d_h,
+                           T_cap, dt, workspace, workspace_bytes, stream, false);
 }
 
 int gqa_out_project(const void *x, const void *W, void *out, int B, int K, int N, gqa_dtype dt,
@@ -536,8 +551,8 @@ int gqa_layer_decode_step(const void *h, const void *W_Q, const void *W_K, const
     void *pws = pbytes ? ws + 2 * qbytes : nullptr;  // split-K projections, when the shape allows them
     uint8_t *dws = ws + 2 * qbytes + pbytes;
     // 1. q = h W_Q; k, v appended at seqlens[b]
-    int rc = gqa_qkv_append(h, W_Q, W_K, W_V, q, k_cache, v_cache, seqlens, seqlens_out, B, d, H, G, d_h, T_cap,
-                            dt, pws, pbytes, stream);
+    int rc = qkv_append_impl(h, W_Q, W_K, W_V, q, k_cache, v_cache, seqlens, seqlens_out, B, d, H, G, d_h,
+                             T_cap, dt, pws, pbytes, stream, true);
     if (rc) return rc;
     // 2. attention over the cache including the new token.  No early L2 warm-up
     //    here: the projection before it streams its weights to the end, and

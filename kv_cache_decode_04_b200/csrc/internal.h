@@ -74,6 +74,7 @@ struct QkvArgs {
     void *workspace;         // null: one CTA per 64-column block; else the split-K kernel
     int num_sms;
     unsigned long long tag;  // nonzero, < 2^32: this call's tag for the split-K block counters
+    int warm;                // nonzero: the column kernel asks L2 for its first weight tiles early
 };
 cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUtensorMap *tk,
                               const CUtensorMap *tv, const CUtensorMap *th, cudaStream_t stream);

@@ -54,6 +54,7 @@ struct ProjParams {
     int nq, nk;               // 64-column blocks of W_Q and of W_K (= of W_V); nk = 0: one weight
     int out_ld;               // row stride of q_out (H*d_h, or N for a single weight)
     unsigned long long timeout_ns;
+    int warm;                 // nonzero: ask L2 for the first weight tiles before the wait
 };
 
 // [128 rows x 64 bf16] tile, 128-byte swizzle: 16-byte chunk ^= row mod 8.
@@ -93,6 +94,13 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         fence_barrier_init();
     }
     __syncthreads();
+    if (p.warm && warp == kCW && lane == 0) {  // L2 hint: the first ring of weight tiles
+        tma_prefetch_desc(tm);
+        for (int kt = 0; kt < min(kStagesP, n_kt); ++kt)
+            asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                             reinterpret_cast<uint64_t>(tm)), "r"(col0), "r"(kt * kKT)
+                         : "memory");
+    }
     pdl_wait_primary();  // h and seqlens written by the kernels before this one are visible
 
     if (warp == kCW) {  // ---------------- TMA producer
@@ -628,6 +636,7 @@ cudaError_t launch_qkv_append(const QkvArgs &a, const CUtensorMap *tq, const CUt
     p.nk = a.G * a.d_h / kNT;
     p.out_ld = a.H * a.d_h;
     p.timeout_ns = a.timeout_ns;
+    p.warm = a.warm;
     return launch_proj(p, a.workspace, a.num_sms, a.tag, tq, tk, tv, th, st);
 }
 
